@@ -1,0 +1,146 @@
+"""fp64 CPU oracle for the DiT attention-block hot path.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline leg may import this package; the product path never does. It shares
+no code with the CUDA library: the arithmetic lives in ``dit3d_oracle.c`` and
+this module only marshals numpy float64 arrays into it.
+
+Each wrapper cites the passage it restates:
+
+* ``adaln_modulate`` / ``gated_residual`` -- "DiT, Flow Matching e 3D Attention",
+  section "A ruptura da U-Net" (adaLN-Zero).
+* ``rope3d`` -- same page, section "3D-RoPE e atencao espaco-temporal".
+* ``attn_fwd`` -- same section, and "Por que e absurdamente dificil gerar um
+  filme inteiro usando IA", section "Matematica por tras".
+* ``patch_grid_tokens`` -- same DiT page, the patchify diagram of section
+  "A ruptura da U-Net": N = (T/p_t)(H/p_h)(W/p_w).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dit3d_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+        lib.oracle_adaln_modulate.argtypes = [P, P, P, P, i64, i32, i64, f64, f64]
+        lib.oracle_gated_residual.argtypes = [P, P, P, P, i64, i32, i64]
+        lib.oracle_rope3d.argtypes = [P, P, i64, i32, i32, P, i32, i32, i32, i32, i32, i32, f64,
+                                      i32, i32, i32]
+        lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, P, i32, f64, P, i64]
+        for f in (lib.oracle_adaln_modulate, lib.oracle_gated_residual, lib.oracle_rope3d,
+                  lib.oracle_attn_fwd):
+            f.restype = None
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _cu(cu_seqlens) -> np.ndarray:
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    assert cu.ndim == 1 and cu[0] == 0 and np.all(np.diff(cu) >= 0)
+    return cu
+
+
+def patch_grid_tokens(T: int, H: int, W: int, p_t: int, p_h: int, p_w: int) -> int:
+    """Number of patch tokens N = (T/p_t)(H/p_h)(W/p_w) of a C x T x H x W latent."""
+    assert T % p_t == 0 and H % p_h == 0 and W % p_w == 0
+    return (T // p_t) * (H // p_h) * (W // p_w)
+
+
+def adaln_modulate(x, gamma, beta, rows_per_group: int, eps: float = 1e-6,
+                   scale_offset: float = 1.0) -> np.ndarray:
+    """u = LayerNorm(x) * (scale_offset + gamma_g) + beta_g, fp64. x: [rows, D]; gamma, beta: [G, D]."""
+    x, gamma, beta = _f64(x), _f64(gamma), _f64(beta)
+    rows, D = x.shape
+    assert rows % rows_per_group == 0 and gamma.shape == beta.shape == (rows // rows_per_group, D)
+    out = np.empty_like(x)
+    _load().oracle_adaln_modulate(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(out), rows, D,
+                                  rows_per_group, eps, scale_offset)
+    return out
+
+
+def gated_residual(x, y, alpha, rows_per_group: int) -> np.ndarray:
+    """out = x + alpha_g * y, fp64. x, y: [rows, D]; alpha: [G, D]."""
+    x, y, alpha = _f64(x), _f64(y), _f64(alpha)
+    rows, D = x.shape
+    assert y.shape == x.shape and alpha.shape == (rows // rows_per_group, D)
+    out = np.empty_like(x)
+    _load().oracle_gated_residual(_ptr(x), _ptr(y), _ptr(alpha), _ptr(out), rows, D,
+                                  rows_per_group)
+    return out
+
+
+def rope3d(v, cu_seqlens, grid_h: int, grid_w: int, bands, base: float = 10000.0,
+           offsets=(0, 0, 0)) -> np.ndarray:
+    """3D-RoPE of v: [rows, H, d] (fp64), positions restarting at every sequence start."""
+    v = _f64(v)
+    rows, H, d = v.shape
+    cu = _cu(cu_seqlens)
+    assert cu[-1] == rows
+    d_t, d_h, d_w = bands
+    assert d_t + d_h + d_w == d and d_t % 2 == 0 and d_h % 2 == 0 and d_w % 2 == 0
+    out = np.empty_like(v)
+    _load().oracle_rope3d(_ptr(v), _ptr(out), rows, H, d, _ptr(cu), len(cu) - 1, grid_h, grid_w,
+                          d_t, d_h, d_w, float(base), *[int(o) for o in offsets])
+    return out
+
+
+def attn_fwd(q, k, v, cu_seqlens, scale: float | None = None, qrows=None, rope=None):
+    """softmax(q k^T * scale) v per sequence and head, fp64.
+
+    q, k, v: [rows, H, d]. ``rope`` (optional) = dict(grid_h, grid_w, bands, base, offsets):
+    q and k are rotated by ``rope3d`` first. ``qrows`` (optional) lists the query rows to
+    compute. Returns (o [n_q, H, d], lse [n_q, H]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    rows, H, d = k.shape
+    cu = _cu(cu_seqlens)
+    assert cu[-1] == rows and q.shape == k.shape == v.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    if rope is not None:
+        q = rope3d(q, cu, **rope)
+        k = rope3d(k, cu, **rope)
+    if qrows is None:
+        n_q, qr_ptr, qr = rows, None, None
+    else:
+        qr = np.ascontiguousarray(qrows, dtype=np.int64)
+        assert qr.min() >= 0 and qr.max() < rows
+        n_q, qr_ptr = len(qr), _ptr(qr)
+    o = np.empty((n_q, H, d), dtype=np.float64)
+    lse = np.empty((n_q, H), dtype=np.float64)
+    _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), rows, H, d, _ptr(cu),
+                            len(cu) - 1, float(scale), qr_ptr, n_q)
+    return o, lse
