@@ -1,0 +1,328 @@
+#!/usr/bin/env python
+"""Benchmark of the DiT attention-block hot path on B200.
+
+One step = one pass of the whole path over one batch of the workload:
+  u   = dit_adaln_modulate(x, gamma, beta)               (adaLN, memory-bound)
+  o   = dit_attn_fwd(q, k, v, rope=3D-RoPE)              (RoPE fused, tensor-core bound)
+  out = dit_gated_residual(x, o, alpha)                  (adaLN-Zero gate, memory-bound)
+The q/k/v projections around the path are not part of it; q, k, v, x and the adaLN
+parameters are seeded synthetic bf16 tensors with the workload's shapes.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p] [--impl reference]
+
+Prints one JSON line (rank 0). `value` is attention TFLOP/s over the whole step
+(algorithmic 4*L^2*d*H FLOPs of every sequence, all ranks, / max-over-ranks time).
+With N > 1 (torchrun), every rank runs its own batch (weak scaling, no collective
+on the data path). `--impl reference` times the fp64 CPU oracle instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
+UNIT = "TFLOP/s"
+# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch from an ncu capture,
+# per query/key token pair and head (scaled to the workload); None until captured.
+ATTN_DRAM_BYTES_PER_LAUNCH = None
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_attention(w, inp, n_rows: int, seed: int = 0):
+    """Time the oracle's 3D-RoPE attention on `n_rows` sampled query rows (all heads, all
+    keys of their sequences). Returns (TFLOP/s, seconds, sample description, threads)."""
+    import oracle
+    from diffusion_transformer_video_b200 import workloads as wl
+    rng = np.random.default_rng([seed, 77])
+    rows = np.sort(rng.choice(w.rows, size=n_rows, replace=False)).astype(np.int64)
+    cu = w.cu_seqlens
+    q, k, v = (wl.bf16_bits_to_f64(inp[n]) for n in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, cu, qrows=rows, rope=w.rope_desc())
+    dt = time.perf_counter() - t0
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+    flops = float(sum(4.0 * (cu[s + 1] - cu[s]) * w.head_dim * w.heads for s in seq_of))
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"{n_rows} query rows x {w.heads} heads of {w.name}, all keys of their sequence, "
+              f"3D-RoPE of full q and k included (fp64, OpenMP)")
+    return flops / dt / 1e12, dt, sample, threads
+
+
+def run_reference(args, rank, world):
+    from diffusion_transformer_video_b200 import workloads as wl
+    if rank != 0:
+        return
+    w = wl.get_workload(args.workload, args.seed)
+    inp = wl.make_inputs(w, args.seed, which=("q", "k", "v"))
+    n_rows = args.ref_rows
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tf, dt, sample, threads = cpu_oracle_attention(w, inp, n_rows, seed=args.seed + i)
+        if i >= args.warmup:
+            vals.append((tf, dt))
+    value = statistics.mean(v for v, _ in vals)
+    ms = 1e3 * statistics.mean(d for _, d in vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded bf16 N(0,1) inputs widened to fp64)",
+            "config": {"workload": w.name, "rows": w.rows, "heads": w.heads,
+                       "head_dim": w.head_dim, "note": w.note},
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": threads,
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="480p")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--ref-rows", type=int, default=24, help="oracle sample rows per step")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from diffusion_transformer_video_b200 import dit3d, workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = wl.get_workload(args.workload, args.seed)
+    # every rank runs its own batch of the workload (seeded per rank)
+    seed = args.seed + 1000 * rank
+    inp = wl.make_inputs(w, seed)
+    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+            for k, v in inp.items()}
+    dev = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+    rows, D, H, d = w.rows, w.d_model, w.heads, w.head_dim
+    rpg = w.rows_per_group
+    desc = dit3d.rope_desc(w.grid_h, w.grid_w, w.bands, w.base)
+    cu = None
+    if w.varlen:
+        cu_host = torch.from_numpy(w.cu_seqlens)
+        cu = (cu_host.cuda(), cu_host)
+    u = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty(rows, H, d, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(b, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dit3d.dit_adaln_modulate(b["x"], b["gamma"], b["beta"], rpg, out=u)
+        if ev is not None:
+            ev[1].record(stream)
+        dit3d.dit_attn_fwd(b["q"], b["k"], b["v"], n_seq=w.n_seq, cu_seqlens=cu, rope=desc,
+                           out=o)
+        if ev is not None:
+            ev[2].record(stream)
+        dit3d.dit_gated_residual(b["x"], o.view(rows, D), b["alpha"], rpg, out=out)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step(dev)
+    torch.cuda.synchronize()
+    dit3d.dit_check_device()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(K):
+            step(dev, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    dit3d.dit_check_device()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    t_mod = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    t_res = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    clocks = clk.summary()
+
+    # end to end: pinned host inputs -> device, the path, result -> pinned host
+    e2e_keys = ("x", "q", "k", "v", "gamma", "beta", "alpha")
+    dev2 = {k: torch.empty_like(dev[k]) for k in e2e_keys}
+    res_host = torch.empty(rows, D, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(host[k].numel() * 2 for k in e2e_keys)
+    d2h = res_host.numel() * 2
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for k in e2e_keys:
+            dev2[k].copy_(host[k], non_blocking=True)
+        step(dev2)
+        res_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+
+    flops = w.attn_flops()
+    ms_step = elapsed_ms / K
+    if world > 1:
+        tt = torch.tensor([ms_step, e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step, e2e_ms = float(tt[0]), float(tt[1])
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    pk = _peaks()
+    att_tflops = flops / (t_att * 1e-3) / 1e12
+    mod_bytes = 4.0 * rows * D
+    res_bytes = 6.0 * rows * D
+    mod_gbs = mod_bytes / (t_mod * 1e-3) / 1e9
+    res_gbs = res_bytes / (t_res * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, sample, threads = cpu_oracle_attention(w, inp, args.cpu_rows, args.seed)
+        cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+               "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded bf16 N(0,1) x/q/k/v, N(0,0.1) adaLN params)",
+            "config": {"workload": w.name, "batch": w.n_seq, "seq_len": w.max_seqlen,
+                       "rows": rows, "heads": H, "head_dim": d, "d_model": D,
+                       "rope_bands": list(w.bands), "grid": [w.grid_h, w.grid_w],
+                       "parallelism": f"dp{world} (independent batches)",
+                       "l2": "inputs larger than L2 (x, q, k, v are %.0f MB each)" % (rows * D * 2 / 1e6)
+                       if rows * D * 2 > 126e6 else "inputs smaller than L2 (no flush)",
+                       "note": w.note},
+            "gpu_launches": 3 * K,
+            "roofline": {"bound": "tensor", "achieved": att_tflops,
+                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": att_tflops / pk["bf16_tflops_sustained"],
+                         "traffic": ATTN_DRAM_BYTES_PER_LAUNCH,
+                         "kernel": "dit_attn_fwd (fused 3D-RoPE)",
+                         "peak_source": f"{pk['source']} sustained bf16 "
+                                        f"(burst {pk['bf16_tflops']}: frac "
+                                        f"{att_tflops / pk['bf16_tflops']:.3f})"},
+            "components": {
+                "adaln_modulate": {"ms": t_mod, "GB/s": mod_gbs, "frac_hbm": mod_gbs / pk["hbm_gbs"],
+                                   "bytes": mod_bytes},
+                "attn_fwd": {"ms": t_att, "TFLOP/s": att_tflops, "flops": flops},
+                "gated_residual": {"ms": t_res, "GB/s": res_gbs, "frac_hbm": res_gbs / pk["hbm_gbs"],
+                                   "bytes": res_bytes},
+            },
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,457 @@
+// Flash-style forward attention with fused 3D-RoPE for sm_100a.
+//
+//   o = softmax(q_rot k_rot^T * scale) v     per (sequence, head), non-causal
+//
+// ("DiT, Flow Matching e 3D Attention", section "3D-RoPE e atencao
+// espaco-temporal"; "Por que e absurdamente dificil gerar um filme inteiro usando
+// IA", section "Matematica por tras". The N x N score matrix never leaves the SM:
+// it lives in tensor memory one 128 x 128 tile at a time.)
+//
+// One CTA computes two 128-row query tiles (Q0, Q1) of one head of one sequence
+// and streams the sequence's keys/values in 128-row tiles through a 2-stage
+// shared-memory ring. 384 threads in three warpgroups:
+//   WG0 (warps 0-3)  softmax of Q0: thread i owns query row i = TMEM lane i.
+//   WG1 (warps 4-7)  softmax of Q1.
+//   warp 8           TMA producer: Q0, Q1 once, then K_j, V_j per stage.
+//   warp 9           TMEM allocator and tcgen05.mma issuer (one thread).
+//   warps 10-11      3D-RoPE: rotate Q0/Q1 and every K_j in shared memory, in
+//                    place, right after TMA lands them (fp32 math, bf16 result).
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
+// O1 [384,384+d). P_i (bf16, two per column) overwrites the first 64 columns of
+// S_i once the softmax has read S_i into registers.
+// MMA order (ping-pong, so one tile's softmax overlaps the other tile's MMAs):
+//   S0=Q0K0, S1=Q1K0, then for each j: O0+=P0V_j, S0=Q0K_{j+1}, O1+=P1V_j, S1=Q1K_{j+1}.
+// Tensor-core operations issued by one thread run in order, and a commit arrives
+// only when every earlier operation of that thread is complete, so when the
+// softmax sees S_i(j+1) the product O_i += P_i(j)V_j has landed and O_i may be
+// rescaled in place.
+// Online softmax in base 2 with a lazily updated row maximum: the running max is
+// only raised (and O, l rescaled) when a new score exceeds it by more than 2^8,
+// which keeps every exponent <= 8 and skips most O rescales.
+// Every mbarrier wait is bounded; on expiry the CTA sets an error bit, drains its
+// in-flight copies and MMAs, frees its tensor memory and exits.
+#pragma once
+#include "common.cuh"
+#include "rope3d.cuh"
+#include "sm100_ptx.cuh"
+
+namespace dit3d {
+namespace attn {
+
+constexpr int kThreads = 384;
+constexpr int kTileM = 128;
+constexpr int kTileN = 128;
+constexpr int kStages = 2;
+constexpr int kRopeThreads = 64;
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpRope0 = 10;
+constexpr uint32_t kTmemCols = 512;
+__host__ __device__ constexpr uint32_t col_s(int qi) { return qi ? 128u : 0u; }
+__host__ __device__ constexpr uint32_t col_o(int qi) { return qi ? 384u : 256u; }
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct Params {
+  const int32_t* cu_seqlens;  // device, n_seq + 1 entries, or nullptr (dense)
+  int32_t n_seq;
+  int64_t dense_len;          // sequence length when cu_seqlens == nullptr
+  int32_t pairs_per_dense_seq;
+  int32_t H;
+  float scale_log2;           // softmax scale * log2(e)
+  __nv_bfloat16* o;
+  float* lse;                 // nullable, [rows, H]
+  int32_t use_rope;
+  RopeParams rope;
+  int32_t force_timeout;
+};
+
+template <int D>
+struct Smem {
+  static constexpr uint32_t kTile = kTileM * D * 2;           // one Q, K or V tile
+  static constexpr uint32_t kQ0 = 0, kQ1 = kTile;
+  static constexpr uint32_t kK = 2 * kTile;                   // + stage * kTile
+  static constexpr uint32_t kV = kK + kStages * kTile;        // + stage * kTile
+  static constexpr uint32_t kBytes = kV + kStages * kTile;
+  // dynamic smem request: forces one CTA per SM (the CTA takes all 512 TMEM columns)
+  static constexpr uint32_t kRequest = (kBytes + 1024 > 120 * 1024) ? kBytes + 1024 : 120 * 1024;
+};
+
+struct Barriers {
+  uint64_t q_full, q_ready;
+  uint64_t k_full[kStages], v_full[kStages], k_ready[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_final, drain;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Byte offset of the 16-byte chunk `cc` (8 bf16) of row r inside a 128-row tile
+// stored as d/64 column blocks of [128 rows x 128 B] with the 128-byte TMA swizzle.
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int cc) {
+  return static_cast<uint32_t>((cc >> 3) * 16384 + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
+}
+
+// Rotate rows [0, n_valid) of one tile in shared memory. Row r of the tile is
+// token (row0 + r) of its sequence. Runs on the kRopeThreads RoPE threads.
+template <int D>
+__device__ __forceinline__ void rope_tile(uint8_t* tile, int64_t row0, int n_valid,
+                                          const RopeParams& rp, int rt, int* s_pos) {
+  constexpr int CPR = D / 8;                 // 16-byte chunks per row
+  constexpr int RPP = kRopeThreads / CPR;    // rows per pass
+  // positions of the tile rows, packed t | h << 11 | w << 22 (host checks the ranges)
+  for (int r = rt; r < kTileM; r += kRopeThreads) {
+    int t = 0, h = 0, w = 0;
+    if (r < n_valid) token_pos(row0 + r, rp.grid_h, rp.grid_w, t, h, w);
+    s_pos[r] = t | (h << 11) | (w << 22);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");
+  const int cc = rt % CPR;
+  PairRef pr[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pr[e] = rope_pair_ref(rp, cc * 4 + e);
+  for (int r = rt / CPR; r < n_valid; r += RPP) {
+    const int pk = s_pos[r];
+    const int t = pk & 2047, h = (pk >> 11) & 2047, w = (pk >> 22) & 1023;
+    uint4* p = reinterpret_cast<uint4*>(tile + sw128_chunk(r, cc));
+    float2 cs[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cs[e] = rope_cs(rp, pr[e], t, h, w);
+    *p = rope_rotate_chunk(*p, cs);
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");  // s_pos reuse
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using L = Smem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ Barriers bars;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ int s_abort;
+  __shared__ int s_pos[kTileM];
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int head = blockIdx.y;
+
+  // ---- work decode: which sequence and which pair of query tiles
+  int64_t seq_start, seq_len;
+  int pair;
+  if (p.cu_seqlens == nullptr) {
+    const int seq = blockIdx.x / p.pairs_per_dense_seq;
+    pair = blockIdx.x - seq * p.pairs_per_dense_seq;
+    seq_len = p.dense_len;
+    seq_start = static_cast<int64_t>(seq) * p.dense_len;
+  } else {
+    int acc = 0, s = 0;
+    pair = 0;
+    seq_start = 0;
+    seq_len = 0;
+    for (; s < p.n_seq; ++s) {
+      const int64_t a = __ldg(p.cu_seqlens + s), b = __ldg(p.cu_seqlens + s + 1);
+      const int np = static_cast<int>((b - a + 2 * kTileM - 1) / (2 * kTileM));
+      if (static_cast<int>(blockIdx.x) < acc + np) {
+        pair = blockIdx.x - acc;
+        seq_start = a;
+        seq_len = b - a;
+        break;
+      }
+      acc += np;
+    }
+  }
+  const int64_t q_row0 = static_cast<int64_t>(pair) * 2 * kTileM;  // within the sequence
+  const int nk = static_cast<int>((seq_len + kTileN - 1) / kTileN);
+  const int last_valid = static_cast<int>(seq_len - static_cast<int64_t>(nk - 1) * kTileN);
+
+  Barriers* b = &bars;
+  volatile int* abort = &s_abort;
+  if (tid == 0) {
+    s_abort = p.force_timeout ? 1 : 0;
+    ptx::mbar_init(ptx::smem_u32(&b->q_full), 1);
+    ptx::mbar_init(ptx::smem_u32(&b->q_ready), kRopeThreads);
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&b->k_full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&b->v_full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&b->k_ready[s]), kRopeThreads);
+      ptx::mbar_init(ptx::smem_u32(&b->kv_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(ptx::smem_u32(&b->s_full[i]), 1);
+      ptx::mbar_init(ptx::smem_u32(&b->p_full[i]), kTileM);
+    }
+    ptx::mbar_init(ptx::smem_u32(&b->o_final), 1);
+    ptx::mbar_init(ptx::smem_u32(&b->drain), 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    ptx::tmem_alloc(ptx::smem_u32(&s_tmem_base), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+
+  if (warp < 8) {
+    // =========================================================== softmax warpgroups
+    const int qi = warp >> 2;
+    const int r = tid & 127;  // query row in tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + col_s(qi);
+    const uint32_t tO = tmem + lane_base + col_o(qi);
+    const uint32_t bar_s = ptx::smem_u32(&b->s_full[qi]);
+    const uint32_t bar_p = ptx::smem_u32(&b->p_full[qi]);
+    float m = -INFINITY;  // running max of scale*log2(e)*score (lazily updated)
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      // warp-uniform decision: tcgen05.ld/st below are warp-collective
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_s, j & 1, abort))) { ok = false; break; }
+      ptx::tc_fence_after();
+      uint32_t sr[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + c * 32, sr + c * 32);
+      ptx::tmem_wait_ld();
+      float* s = reinterpret_cast<float*>(sr);
+      if (j == nk - 1 && last_valid < kTileN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= last_valid) s[c] = -INFINITY;
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float mcand = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+      const bool raise = mcand > m + kRescaleThreshold;
+      if (__any_sync(0xffffffffu, raise && j > 0)) {
+        // warp-collective O rescale (lanes that keep their max use factor 1)
+        const float f = raise ? ex2(m - mcand) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tO + c * 32, ov);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          ptx::tmem_st32(tO + c * 32, ov);
+        }
+        l *= f;
+      }
+      if (raise) m = mcand;
+      const float neg_m = -m;
+      float l0 = 0.f, l1 = 0.f;
+      uint32_t pw[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float e0 = ex2(fmaf(s[2 * c], p.scale_log2, neg_m));
+        const float e1 = ex2(fmaf(s[2 * c + 1], p.scale_log2, neg_m));
+        l0 += e0;
+        l1 += e1;
+        pw[c] = pack_bf16x2(e0, e1);
+      }
+      l += l0 + l1;
+      ptx::tmem_st32(tS, pw);
+      ptx::tmem_st32(tS + 32, pw + 32);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar_p);
+    }
+    // ---- epilogue: O / l -> bf16 -> global, plus the log-sum-exp
+    if (__all_sync(0xffffffffu, ok && ptx::mbar_wait(ptx::smem_u32(&b->o_final), 0, abort))) {
+      ptx::tc_fence_after();
+      const int64_t row_in_seq = q_row0 + qi * kTileM + r;
+      const bool valid = row_in_seq < seq_len;
+      const float inv_l = 1.f / l;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
+                      ((seq_start + row_in_seq) * p.H + head) * static_cast<int64_t>(D) * 2;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        ptx::tmem_ld32(tO + c * 32, ov);
+        ptx::tmem_wait_ld();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l,
+                                __uint_as_float(ov[2 * e + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr)
+        p.lse[(seq_start + row_in_seq) * p.H + head] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+  } else if (warp == kWarpTma) {
+    // =========================================================== TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_q);
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_v);
+      const int x0 = head * D;
+      const uint32_t q_full = ptx::smem_u32(&b->q_full);
+      int issued = 0;  // K/V tiles issued
+      if (!*abort) {
+        ptx::mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+        for (int qi = 0; qi < 2; ++qi)
+          for (int blk = 0; blk < D / 64; ++blk)
+            ptx::tma_load_2d(ptx::smem_u32(smem + (qi ? L::kQ1 : L::kQ0) + blk * 16384), &tm_q,
+                             x0 + blk * 64, static_cast<int>(seq_start + q_row0 + qi * kTileM),
+                             q_full);
+        for (int j = 0; j < nk; ++j) {
+          const int st = j % kStages;
+          if (j >= kStages &&
+              !ptx::mbar_wait(ptx::smem_u32(&b->kv_empty[st]), ((j / kStages) - 1) & 1, abort))
+            break;
+          const int y = static_cast<int>(seq_start + static_cast<int64_t>(j) * kTileN);
+          const uint32_t kf = ptx::smem_u32(&b->k_full[st]), vf = ptx::smem_u32(&b->v_full[st]);
+          ptx::mbar_arrive_expect_tx(kf, L::kTile);
+          for (int blk = 0; blk < D / 64; ++blk)
+            ptx::tma_load_2d(ptx::smem_u32(smem + L::kK + st * L::kTile + blk * 16384), &tm_k,
+                             x0 + blk * 64, y, kf);
+          ptx::mbar_arrive_expect_tx(vf, L::kTile);
+          for (int blk = 0; blk < D / 64; ++blk)
+            ptx::tma_load_2d(ptx::smem_u32(smem + L::kV + st * L::kTile + blk * 16384), &tm_v,
+                             x0 + blk * 64, y, vf);
+          ++issued;
+        }
+        // drain: no copy may still be in flight into shared memory when the CTA exits
+        // (normally these phases completed long ago and the waits return at once)
+        volatile int never = 0;
+        ptx::mbar_wait(q_full, 0, &never);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+          const int st = j % kStages;
+          ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), (j / kStages) & 1, &never);
+          ptx::mbar_wait(ptx::smem_u32(&b->v_full[st]), (j / kStages) & 1, &never);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = ptx::make_idesc_bf16_f32(kTileM, kTileN, false);
+      constexpr uint32_t idesc_pv = ptx::make_idesc_bf16_f32(kTileM, D, true);
+      const uint32_t sbase = ptx::smem_u32(smem);
+      bool issued_any = false;
+      auto qk = [&](int qi, int st) {
+        const uint32_t qa = sbase + (qi ? L::kQ1 : L::kQ0);
+        const uint32_t ka = sbase + L::kK + st * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::umma_ss(tmem + col_s(qi), ptx::make_smem_desc(qa + off, 16, 1024, ptx::kSwizzle128B),
+                       ptx::make_smem_desc(ka + off, 16, 1024, ptx::kSwizzle128B), idesc_qk,
+                       kk > 0);
+        }
+        ptx::umma_commit(ptx::smem_u32(&b->s_full[qi]));
+      };
+      auto pv = [&](int qi, int st, bool acc) {
+        const uint32_t va = sbase + L::kV + st * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          ptx::umma_ts(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
+                       ptx::make_smem_desc(va + kk * 2048, 16384, 1024, ptx::kSwizzle128B),
+                       idesc_pv, (acc || kk > 0) ? 1u : 0u);
+      };
+      const uint32_t q_wait = ptx::smem_u32(p.use_rope ? &b->q_ready : &b->q_full);
+      bool ok = ptx::mbar_wait(q_wait, 0, abort);
+      if (ok) ok = ptx::mbar_wait(ptx::smem_u32(p.use_rope ? &b->k_ready[0] : &b->k_full[0]), 0, abort);
+      if (ok) {
+        ptx::tc_fence_after();
+        qk(0, 0);
+        qk(1, 0);
+        issued_any = true;
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int st = j % kStages, ph = (j / kStages) & 1;
+        const int st1 = (j + 1) % kStages, ph1 = ((j + 1) / kStages) & 1;
+        const bool more = j + 1 < nk;
+        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[st]), ph, abort))) break;
+        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->p_full[0]), j & 1, abort))) break;
+        ptx::tc_fence_after();
+        pv(0, st, j > 0);
+        if (more) {
+          if (!(ok = ptx::mbar_wait(
+                    ptx::smem_u32(p.use_rope ? &b->k_ready[st1] : &b->k_full[st1]), ph1, abort)))
+            break;
+          ptx::tc_fence_after();
+          qk(0, st1);
+        }
+        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->p_full[1]), j & 1, abort))) break;
+        ptx::tc_fence_after();
+        pv(1, st, j > 0);
+        ptx::umma_commit(ptx::smem_u32(&b->kv_empty[st]));
+        if (more) qk(1, st1);
+      }
+      if (ok) ptx::umma_commit(ptx::smem_u32(&b->o_final));
+      if (issued_any) {
+        // all MMAs of this CTA complete before tensor memory is released
+        volatile int never = 0;
+        ptx::umma_commit(ptx::smem_u32(&b->drain));
+        ptx::mbar_wait(ptx::smem_u32(&b->drain), 0, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // =========================================================== 3D-RoPE warps
+    if (p.use_rope) {
+      const int rt = tid - kWarpRope0 * 32;
+      // every RoPE thread waits itself (acquiring the TMA data), then all 64 agree
+      // before the named barriers inside rope_tile
+      auto all_ok = [](bool ok) {
+        uint32_t r;
+        asm volatile(
+            "{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\t"
+            "bar.red.and.pred b, 2, %2, a;\n\tselp.u32 %0, 1, 0, b;\n\t}"
+            : "=r"(r)
+            : "r"(static_cast<uint32_t>(ok)), "n"(kRopeThreads)
+            : "memory");
+        return r != 0;
+      };
+      if (all_ok(ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort))) {
+        for (int qi = 0; qi < 2; ++qi) {
+          const int64_t r0 = q_row0 + qi * kTileM;
+          const int64_t rem = seq_len - r0;
+          const int nv = rem <= 0 ? 0 : (rem >= kTileM ? kTileM : static_cast<int>(rem));
+          rope_tile<D>(smem + (qi ? L::kQ1 : L::kQ0), r0, nv, p.rope, rt, s_pos);
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
+        for (int j = 0; j < nk; ++j) {
+          const int st = j % kStages, ph = (j / kStages) & 1;
+          if (!all_ok(ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort))) break;
+          const int nv = (j == nk - 1) ? last_valid : kTileN;
+          rope_tile<D>(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv, p.rope,
+                       rt, s_pos);
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(ptx::smem_u32(&b->k_ready[st]));
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort) atomicOr(&g_device_error, kDevErrTimeout);
+  if (warp == kWarpMma) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn
+}  // namespace dit3d

@@ -1,0 +1,387 @@
+// C ABI of libdit3d (declared in include/dit3d.h): argument validation, tensor
+// maps, the RoPE cos/sin table cache and kernel launches. All device work is in
+// the kernels of adaln.cuh, rope3d.cuh and attn_fwd.cuh.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "../../include/dit3d.h"
+#include "adaln.cuh"
+#include "attn_fwd.cuh"
+#include "common.cuh"
+#include "rope3d.cuh"
+
+using namespace dit3d;
+
+namespace {
+
+std::mutex g_mu;
+int g_force_timeout = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// sm_100 check, cached per device.
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_DEVICE;
+  static std::map<int, int> ok_cache;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = ok_cache.find(dev);
+  if (it == ok_cache.end()) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return DIT_ERR_DEVICE;
+    it = ok_cache.emplace(dev, major == 10 ? DIT_OK : DIT_ERR_DEVICE).first;
+  }
+  return it->second;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_LAUNCH; }
+
+int check_rows_groups(int64_t rows, int32_t D, int64_t rows_per_group) {
+  if (rows < 0 || D <= 0 || (D % 8) != 0 || rows_per_group <= 0 || (rows % rows_per_group) != 0)
+    return DIT_ERR_SHAPE;
+  if (rows > INT32_MAX) return DIT_ERR_SHAPE;  // one CTA per row
+  return DIT_OK;
+}
+
+// Sequence layout shared by RoPE and attention: fills the host copy of the lengths.
+int check_seqs(int64_t rows, int32_t n_seq, const int32_t* cu_dev, const int32_t* cu_host,
+               std::vector<int64_t>* lens) {
+  if (n_seq <= 0) return DIT_ERR_SHAPE;
+  lens->clear();
+  if (cu_dev == nullptr && cu_host == nullptr) {
+    if (rows % n_seq != 0) return DIT_ERR_SHAPE;
+    lens->assign(n_seq, rows / n_seq);
+    return DIT_OK;
+  }
+  if (cu_dev == nullptr || cu_host == nullptr) return DIT_ERR_NULL;
+  if (cu_host[0] != 0 || cu_host[n_seq] != rows) return DIT_ERR_SEQLENS;
+  for (int s = 0; s < n_seq; ++s) {
+    if (cu_host[s + 1] < cu_host[s]) return DIT_ERR_SEQLENS;
+    lens->push_back(static_cast<int64_t>(cu_host[s + 1]) - cu_host[s]);
+  }
+  return DIT_OK;
+}
+
+// ---------------------------------------------------------------- RoPE tables
+struct TableKey {
+  int dev, gh, gw, dt, dh, dw, t_ext, t0, h0, w0;
+  uint32_t base_bits;
+  bool operator<(const TableKey& o) const {
+    return std::tie(dev, gh, gw, dt, dh, dw, t_ext, t0, h0, w0, base_bits) <
+           std::tie(o.dev, o.gh, o.gw, o.dt, o.dh, o.dw, o.t_ext, o.t0, o.h0, o.w0, o.base_bits);
+  }
+};
+std::map<TableKey, float2*> g_tables;
+
+int validate_rope(const dit_rope3d_desc* r, int32_t d, const std::vector<int64_t>& lens,
+                  int* t_ext) {
+  if (r->grid_h < 1 || r->grid_w < 1 || r->grid_h > 2047 || r->grid_w > 1023) return DIT_ERR_SHAPE;
+  if (r->d_t < 0 || r->d_h < 0 || r->d_w < 0 || (r->d_t | r->d_h | r->d_w) & 1) return DIT_ERR_SHAPE;
+  if (r->d_t + r->d_h + r->d_w != d) return DIT_ERR_SHAPE;
+  if (!(r->base > 1.0f) || !std::isfinite(r->base)) return DIT_ERR_SHAPE;
+  if (r->t0 < 0 || r->h0 < 0 || r->w0 < 0) return DIT_ERR_SHAPE;
+  const int64_t fr = static_cast<int64_t>(r->grid_h) * r->grid_w;
+  int64_t tmax = 1;
+  for (int64_t L : lens) {
+    if (L % fr != 0) return DIT_ERR_SHAPE;
+    tmax = std::max<int64_t>(tmax, L / fr);
+  }
+  if (tmax > 2047) return DIT_ERR_SHAPE;
+  *t_ext = static_cast<int>((tmax + 31) / 32 * 32);  // round up: fewer distinct tables
+  return DIT_OK;
+}
+
+// Host fp64 -> fp32 (cos, sin) table for the angle (pos + offset) * base^(-2i/d_a).
+int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopeParams* rp) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  uint32_t bb;
+  std::memcpy(&bb, &r->base, 4);
+  TableKey key{dev, r->grid_h, r->grid_w, r->d_t, r->d_h, r->d_w, t_ext, r->t0, r->h0, r->w0, bb};
+  rp->grid_h = r->grid_h;
+  rp->grid_w = r->grid_w;
+  rp->d_t = r->d_t;
+  rp->d_h = r->d_h;
+  rp->d_w = r->d_w;
+  rp->off_h = t_ext * (r->d_t / 2);
+  rp->off_w = rp->off_h + r->grid_h * (r->d_h / 2);
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_tables.find(key);
+  if (it != g_tables.end()) {
+    rp->table = it->second;
+    return DIT_OK;
+  }
+  const int n = rp->off_w + r->grid_w * (r->d_w / 2);
+  std::vector<float2> host(std::max(n, 1));
+  const int ext[3] = {t_ext, r->grid_h, r->grid_w};
+  const int width[3] = {r->d_t, r->d_h, r->d_w};
+  const int off[3] = {r->t0, r->h0, r->w0};
+  int at = 0;
+  for (int a = 0; a < 3; ++a)
+    for (int pos = 0; pos < ext[a]; ++pos)
+      for (int i = 0; i < width[a] / 2; ++i) {
+        const double theta = std::pow(static_cast<double>(r->base), -2.0 * i / width[a]);
+        const double phi = static_cast<double>(pos + off[a]) * theta;
+        host[at++] = make_float2(static_cast<float>(std::cos(phi)), static_cast<float>(std::sin(phi)));
+      }
+  float2* dptr = nullptr;
+  if (cudaMalloc(&dptr, sizeof(float2) * host.size()) != cudaSuccess) return DIT_ERR_ALLOC;
+  // pageable source: the copy has consumed `host` when the call returns
+  if (cudaMemcpyAsync(dptr, host.data(), sizeof(float2) * host.size(), cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess) {
+    cudaFree(dptr);
+    return DIT_ERR_LAUNCH;
+  }
+  g_tables.emplace(key, dptr);
+  rp->table = dptr;
+  return DIT_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// [rows, H*d] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32_t H,
+                const attn::Params& prm, int n_work, cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, static_cast<int64_t>(H) * D) ||
+      !make_tmap(&tk, k, rows, static_cast<int64_t>(H) * D) ||
+      !make_tmap(&tv, v, rows, static_cast<int64_t>(H) * D))
+    return DIT_ERR_LAUNCH;
+  constexpr uint32_t smem = attn::Smem<D>::kRequest;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(attn::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return DIT_ERR_LAUNCH;
+    attr_set[dev] = true;
+  }
+  dim3 grid(n_work, H);
+  attn::attn_fwd_kernel<D><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
+  return launch_status();
+}
+
+template <int NV>
+void launch_modulate(const void* x, const void* g, const void* b, void* o, int64_t rows, int32_t D,
+                     int64_t rpg, float eps, float s0, cudaStream_t st) {
+  adaln_modulate_kernel<NV><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
+      static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
+}
+
+template <int NV>
+void launch_residual(const void* x, const void* y, const void* a, void* o, int64_t rows, int32_t D,
+                     int64_t rpg, cudaStream_t st) {
+  gated_residual_kernel<NV><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y),
+      static_cast<const __nv_bfloat16*>(a), static_cast<__nv_bfloat16*>(o), D, rpg);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dit_status_string(int status) {
+  switch (status) {
+    case DIT_OK: return "DIT_OK";
+    case DIT_ERR_NULL: return "DIT_ERR_NULL: a required pointer is NULL";
+    case DIT_ERR_SHAPE: return "DIT_ERR_SHAPE: unsupported or inconsistent sizes";
+    case DIT_ERR_ALIGN: return "DIT_ERR_ALIGN: a device pointer is not 16-byte aligned";
+    case DIT_ERR_SEQLENS: return "DIT_ERR_SEQLENS: invalid cu_seqlens";
+    case DIT_ERR_DEVICE: return "DIT_ERR_DEVICE: current device is not sm_100";
+    case DIT_ERR_LAUNCH: return "DIT_ERR_LAUNCH: a CUDA call or kernel launch failed";
+    case DIT_ERR_TIMEOUT: return "DIT_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case DIT_ERR_ALLOC: return "DIT_ERR_ALLOC: device allocation for the RoPE table failed";
+    default: return "unknown dit_status";
+  }
+}
+
+int dit_adaln_modulate(const void* x, const void* gamma, const void* beta, void* out, int64_t rows,
+                       int32_t D, int64_t rows_per_group, float eps, float scale_offset,
+                       void* stream) {
+  if (!x || !gamma || !beta || !out) return DIT_ERR_NULL;
+  if (int s = check_rows_groups(rows, D, rows_per_group)) return s;
+  if (!(eps >= 0.f) || !std::isfinite(scale_offset)) return DIT_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(out)) return DIT_ERR_ALIGN;
+  if (int s = check_device()) return s;
+  if (rows == 0) return DIT_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  const int nv = (D / 8 + kRowThreads - 1) / kRowThreads;
+  switch (nv) {
+    case 1: launch_modulate<1>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 2: launch_modulate<2>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 3: launch_modulate<3>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 4: launch_modulate<4>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 5: launch_modulate<5>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 6: launch_modulate<6>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 7: launch_modulate<7>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    case 8: launch_modulate<8>(x, gamma, beta, out, rows, D, rows_per_group, eps, scale_offset, st); break;
+    default:
+      adaln_modulate_wide_kernel<<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gamma),
+          static_cast<const __nv_bfloat16*>(beta), static_cast<__nv_bfloat16*>(out), D,
+          rows_per_group, eps, scale_offset);
+  }
+  return launch_status();
+}
+
+int dit_gated_residual(const void* x, const void* y, const void* alpha, void* out, int64_t rows,
+                       int32_t D, int64_t rows_per_group, void* stream) {
+  if (!x || !y || !alpha || !out) return DIT_ERR_NULL;
+  if (int s = check_rows_groups(rows, D, rows_per_group)) return s;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(alpha) || !aligned16(out)) return DIT_ERR_ALIGN;
+  if (int s = check_device()) return s;
+  if (rows == 0) return DIT_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  const int nv = (D / 8 + kRowThreads - 1) / kRowThreads;
+  switch (nv) {
+    case 1: launch_residual<1>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 2: launch_residual<2>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 3: launch_residual<3>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 4: launch_residual<4>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 5: launch_residual<5>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 6: launch_residual<6>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 7: launch_residual<7>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    case 8: launch_residual<8>(x, y, alpha, out, rows, D, rows_per_group, st); break;
+    default:
+      gated_residual_wide_kernel<<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y),
+          static_cast<const __nv_bfloat16*>(alpha), static_cast<__nv_bfloat16*>(out), D,
+          rows_per_group);
+  }
+  return launch_status();
+}
+
+int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,
+                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                  const int32_t* cu_seqlens_host, const dit_rope3d_desc* rope, void* stream) {
+  if (!q_in || !q_out || !rope || (k_in && !k_out)) return DIT_ERR_NULL;
+  if (rows < 0 || H <= 0 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
+  if (!aligned16(q_in) || !aligned16(q_out) || (k_in && (!aligned16(k_in) || !aligned16(k_out))))
+    return DIT_ERR_ALIGN;
+  std::vector<int64_t> lens;
+  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
+  int t_ext = 0;
+  if (int s = validate_rope(rope, d, lens, &t_ext)) return s;
+  if (int s = check_device()) return s;
+  if (rows == 0) return DIT_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  RopeParams rp;
+  if (int s = get_table(rope, t_ext, st, &rp)) return s;
+  const int64_t dense_len = cu_seqlens_dev ? 0 : rows / n_seq;
+  const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+  if (d == 128)
+    rope3d_qk_kernel<128><<<grid, 256, 0, st>>>(
+        static_cast<const uint4*>(q_in), static_cast<const uint4*>(k_in), static_cast<uint4*>(q_out),
+        static_cast<uint4*>(k_out), rows, H, cu_seqlens_dev, n_seq, dense_len, rp);
+  else
+    rope3d_qk_kernel<64><<<grid, 256, 0, st>>>(
+        static_cast<const uint4*>(q_in), static_cast<const uint4*>(k_in), static_cast<uint4*>(q_out),
+        static_cast<uint4*>(k_out), rows, H, cu_seqlens_dev, n_seq, dense_len, rp);
+  return launch_status();
+}
+
+int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t rows,
+                 int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                 const int32_t* cu_seqlens_host, float softmax_scale, const dit_rope3d_desc* rope,
+                 void* stream) {
+  if (!q || !k || !v || !o) return DIT_ERR_NULL;
+  if (rows <= 0 || H <= 0 || H > 65535 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
+  if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;  // TMA row coordinates are int32
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return DIT_ERR_ALIGN;
+  std::vector<int64_t> lens;
+  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
+  int t_ext = 0;
+  if (rope)
+    if (int s = validate_rope(rope, d, lens, &t_ext)) return s;
+  if (int s = check_device()) return s;
+  auto st = static_cast<cudaStream_t>(stream);
+
+  attn::Params prm{};
+  prm.cu_seqlens = cu_seqlens_dev;
+  prm.n_seq = n_seq;
+  prm.H = H;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.force_timeout = g_force_timeout;
+  int64_t n_work = 0;
+  if (cu_seqlens_dev == nullptr) {
+    prm.dense_len = rows / n_seq;
+    prm.pairs_per_dense_seq = static_cast<int32_t>((prm.dense_len + 2 * attn::kTileM - 1) / (2 * attn::kTileM));
+    n_work = static_cast<int64_t>(prm.pairs_per_dense_seq) * n_seq;
+  } else {
+    for (int64_t L : lens) n_work += (L + 2 * attn::kTileM - 1) / (2 * attn::kTileM);
+  }
+  if (n_work == 0) return DIT_OK;
+  if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
+  if (rope) {
+    prm.use_rope = 1;
+    if (int s = get_table(rope, t_ext, st, &prm.rope)) return s;
+  }
+  if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+  return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+}
+
+int dit_check_device(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DIT_ERR_LAUNCH;
+  uint32_t err = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&err, g_device_error, sizeof(err)) != cudaSuccess) return DIT_ERR_LAUNCH;
+  if (err != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+    return DIT_ERR_LAUNCH;
+  return (err & kDevErrTimeout) ? DIT_ERR_TIMEOUT : DIT_OK;
+}
+
+void dit_shutdown(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_tables) {
+    cudaSetDevice(kv.first.dev);
+    cudaFree(kv.second);
+  }
+  g_tables.clear();
+  cudaSetDevice(cur);
+}
+
+void dit_debug_force_timeout(int enable) { g_force_timeout = enable ? 1 : 0; }
+
+}  // extern "C"

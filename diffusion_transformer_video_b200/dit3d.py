@@ -1,0 +1,191 @@
+"""Thin ctypes binding of libdit3d (include/dit3d.h).
+
+Argument marshalling only: torch tensors become device pointers, the current
+torch CUDA stream becomes the call's stream, and a non-zero status becomes a
+``DitError``. Every computation runs in the library's CUDA kernels; there is no
+fallback. The functions carry the C names.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdit3d.so")
+
+DIT_OK = 0
+STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_ALIGN",
+                4: "DIT_ERR_SEQLENS", 5: "DIT_ERR_DEVICE", 6: "DIT_ERR_LAUNCH",
+                7: "DIT_ERR_TIMEOUT", 8: "DIT_ERR_ALLOC"}
+
+# every symbol include/dit3d.h declares
+EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
+           "dit_check_device", "dit_status_string", "dit_shutdown", "dit_debug_force_timeout")
+
+
+class DitError(RuntimeError):
+    def __init__(self, status: int, lib):
+        self.status = status
+        super().__init__(lib.dit_status_string(status).decode())
+
+
+class RopeDesc(ctypes.Structure):
+    """dit_rope3d_desc: patch grid, band widths (t|h|w), frequency base, position offsets."""
+    _fields_ = [("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("d_t", ctypes.c_int32), ("d_h", ctypes.c_int32), ("d_w", ctypes.c_int32),
+                ("base", ctypes.c_float),
+                ("t0", ctypes.c_int32), ("h0", ctypes.c_int32), ("w0", ctypes.c_int32)]
+
+
+def rope_desc(grid_h, grid_w, bands, base=10000.0, offsets=(0, 0, 0)) -> RopeDesc:
+    return RopeDesc(int(grid_h), int(grid_w), int(bands[0]), int(bands[1]), int(bands[2]),
+                    float(base), int(offsets[0]), int(offsets[1]), int(offsets[2]))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m "
+                               "diffusion_transformer_video_b200.build` (there is no fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+        L.dit_adaln_modulate.argtypes = [P, P, P, P, i64, i32, i64, f32, f32, P]
+        L.dit_gated_residual.argtypes = [P, P, P, P, i64, i32, i64, P]
+        L.dit_rope3d_qk.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
+                                    ctypes.POINTER(RopeDesc), P]
+        L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
+                                   ctypes.POINTER(RopeDesc), P]
+        L.dit_check_device.argtypes = [P]
+        L.dit_status_string.argtypes = [ctypes.c_int]
+        L.dit_status_string.restype = ctypes.c_char_p
+        L.dit_shutdown.argtypes = []
+        L.dit_shutdown.restype = None
+        L.dit_debug_force_timeout.argtypes = [ctypes.c_int]
+        L.dit_debug_force_timeout.restype = None
+        for name in ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
+                     "dit_check_device"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != DIT_OK:
+        raise DitError(status, lib())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _bf16(t: torch.Tensor, name: str):
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+
+
+def _keep(cu_dev):
+    # a device copy made here must outlive the kernel that reads it
+    if cu_dev is not None:
+        cu_dev.record_stream(torch.cuda.current_stream())
+
+
+def _cu_args(cu_seqlens):
+    """(device tensor, host tensor, n_seq) for a packed layout, or Nones for dense.
+
+    ``cu_seqlens`` is a host sequence/tensor of n_seq + 1 int32 prefix sums, or a
+    ``(device_tensor, host_tensor)`` pair prepared once by the caller."""
+    if cu_seqlens is None:
+        return None, None, None
+    if isinstance(cu_seqlens, tuple):
+        dev, host = cu_seqlens
+        return dev, host, host.numel() - 1
+    if isinstance(cu_seqlens, torch.Tensor):
+        host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+    else:
+        host = torch.as_tensor(cu_seqlens, dtype=torch.int32).contiguous()
+    dev = host.to("cuda", non_blocking=False)
+    return dev, host, host.numel() - 1
+
+
+def dit_adaln_modulate(x, gamma, beta, rows_per_group, out=None, eps=1e-6, scale_offset=1.0):
+    """out = LayerNorm(x) * (scale_offset + gamma_g) + beta_g (x: [rows, D] bf16)."""
+    for t, n in ((x, "x"), (gamma, "gamma"), (beta, "beta")):
+        _bf16(t, n)
+    out = torch.empty_like(x) if out is None else out
+    _bf16(out, "out")
+    rows, D = x.shape[0], x.shape[-1]
+    _check(lib().dit_adaln_modulate(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(out), rows, D,
+                                    int(rows_per_group), float(eps), float(scale_offset),
+                                    _stream()))
+    return out
+
+
+def dit_gated_residual(x, y, alpha, rows_per_group, out=None):
+    """out = x + alpha_g * y (all [rows, D] bf16; alpha [G, D])."""
+    for t, n in ((x, "x"), (y, "y"), (alpha, "alpha")):
+        _bf16(t, n)
+    out = torch.empty_like(x) if out is None else out
+    _bf16(out, "out")
+    rows, D = x.shape[0], x.shape[-1]
+    _check(lib().dit_gated_residual(_ptr(x), _ptr(y), _ptr(alpha), _ptr(out), rows, D,
+                                    int(rows_per_group), _stream()))
+    return out
+
+
+def dit_rope3d_qk(q, k, rope: RopeDesc, n_seq=1, cu_seqlens=None, q_out=None, k_out=None,
+                  inplace=False):
+    """3D-RoPE of q and k ([rows, H, d] bf16). Returns (q_rot, k_rot)."""
+    _bf16(q, "q")
+    if k is not None:
+        _bf16(k, "k")
+    if inplace:
+        q_out, k_out = q, k
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    if k is not None:
+        k_out = torch.empty_like(k) if k_out is None else k_out
+    rows, H, d = q.shape
+    cu_dev, cu_host, ns = _cu_args(cu_seqlens)
+    n = ns if ns is not None else n_seq
+    _check(lib().dit_rope3d_qk(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), rows, H, d, n,
+                               _ptr(cu_dev), _ptr(cu_host), ctypes.byref(rope), _stream()))
+    _keep(cu_dev)
+    return q_out, k_out
+
+
+def dit_attn_fwd(q, k, v, n_seq=1, cu_seqlens=None, rope: RopeDesc | None = None,
+                 softmax_scale=0.0, out=None, return_lse=False):
+    """softmax(q_rot k_rot^T * scale) v per sequence and head ([rows, H, d] bf16)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n)
+    rows, H, d = q.shape
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((rows, H), dtype=torch.float32, device=q.device) if return_lse else None
+    cu_dev, cu_host, ns = _cu_args(cu_seqlens)
+    n = ns if ns is not None else n_seq
+    _check(lib().dit_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), rows, H, d, n,
+                              _ptr(cu_dev), _ptr(cu_host), float(softmax_scale),
+                              ctypes.byref(rope) if rope is not None else None, _stream()))
+    _keep(cu_dev)
+    return (out, lse) if return_lse else out
+
+
+def dit_check_device():
+    """Synchronises the current stream and raises DitError if a kernel gave up a wait."""
+    _check(lib().dit_check_device(_stream()))
+
+
+def dit_shutdown():
+    lib().dit_shutdown()

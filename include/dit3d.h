@@ -1,0 +1,143 @@
+/*
+ * dit3d.h -- C ABI of libdit3d: the hot path of a video Diffusion Transformer
+ * block on NVIDIA B200 (sm_100a).
+ *
+ *   u   = LayerNorm(x) * (s0 + gamma_g) + beta_g            dit_adaln_modulate
+ *   q,k = R3D(t, h, w) q,  R3D(t, h, w) k                     dit_rope3d_qk
+ *   o   = softmax(q_rot k_rot^T / sqrt(d_head)) v             dit_attn_fwd
+ *   out = x + alpha_g * y                                     dit_gated_residual
+ *
+ * Formulas: "DiT, Flow Matching e 3D Attention: A Engenharia de Video com IA",
+ * sections "A ruptura da U-Net" (adaLN-Zero) and "3D-RoPE e atencao
+ * espaco-temporal" (band split of the head dimension, rotated q/k, attention);
+ * "Por que e absurdamente dificil gerar um filme inteiro usando IA", section
+ * "Matematica por tras" (softmax(QK^T/sqrt(d))V).
+ *
+ * Conventions shared by every call
+ *  - Tensors are dense, row-major, token-major bf16 in device memory, with no
+ *    strides: activations [rows, D]; q/k/v/o [rows, H, d] (= [rows, D], D = H*d).
+ *  - Every device pointer must be 16-byte aligned (128-bit loads and TMA).
+ *  - The caller owns every buffer. Calls allocate nothing per call; the RoPE
+ *    cos/sin tables (fp64 on the host, stored fp32) are cached in device memory
+ *    per (device, descriptor, extent) on first use and freed by dit_shutdown().
+ *    Make the first call for a given RoPE descriptor outside CUDA-graph capture.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only enqueue
+ *    work: they return before the GPU has run it. Validation reads host data only.
+ *  - Return value: DIT_OK or a dit_status code; nothing is printed, thrown or
+ *    exited. Nothing is launched when validation fails.
+ *  - Sequence layout (RoPE and attention). Dense: cu_seqlens_* = NULL and the
+ *    rows form n_seq equal sequences of rows / n_seq tokens. Packed (varlen):
+ *    cu_seqlens_host and cu_seqlens_dev both hold the same n_seq + 1 int32
+ *    exclusive prefix sums (cu[0] = 0, non-decreasing, cu[n_seq] = rows).
+ *  - Token order inside a sequence: row-major over the patch grid, t slowest,
+ *    w fastest: token j has w = j % grid_w, h = (j / grid_w) % grid_h,
+ *    t = j / (grid_h * grid_w). Positions restart at 0 for every sequence.
+ */
+#ifndef DIT3D_H_
+#define DIT3D_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum dit_status {
+  DIT_OK = 0,
+  DIT_ERR_NULL = 1,     /* a required pointer is NULL                                  */
+  DIT_ERR_SHAPE = 2,    /* unsupported or inconsistent sizes (see each call)            */
+  DIT_ERR_ALIGN = 3,    /* a device pointer is not 16-byte aligned                      */
+  DIT_ERR_SEQLENS = 4,  /* cu_seqlens not 0-based, decreasing, or not ending at rows    */
+  DIT_ERR_DEVICE = 5,   /* current device is not sm_100 (B200 class)                     */
+  DIT_ERR_LAUNCH = 6,   /* a CUDA call or kernel launch failed                          */
+  DIT_ERR_TIMEOUT = 7,  /* a kernel's bounded wait expired (reported by dit_check_device) */
+  DIT_ERR_ALLOC = 8     /* the RoPE table cache could not allocate device memory        */
+};
+
+/* 3D-RoPE descriptor (DiT page, section "3D-RoPE e atencao espaco-temporal"):
+ * the head dimension is cut into contiguous bands [t | h | w] of widths d_t, d_h,
+ * d_w (each even, d_t + d_h + d_w = head_dim). In band a, the pair
+ * (v[o_a+2i], v[o_a+2i+1]) turns by pos_a * base^(-2i/d_a) with the rotation
+ * [[cos, -sin], [sin, cos]]; pos_a is the token's patch coordinate plus the
+ * offset (t0, h0, w0). The frequency law, base and pair layout are this
+ * library's reading: the pages give only the band split. */
+typedef struct dit_rope3d_desc {
+  int32_t grid_h, grid_w; /* patch-grid height H_lat/p_h and width W_lat/p_w (>= 1)      */
+  int32_t d_t, d_h, d_w;  /* band widths, even, summing to head_dim                        */
+  float base;             /* frequency base, > 1 (10000 in the workloads)                  */
+  int32_t t0, h0, w0;     /* position offsets added to every token (>= 0)                   */
+} dit_rope3d_desc;
+
+/* adaLN modulation before attention or MLP (DiT page, "A ruptura da U-Net"):
+ *   out[r, c] = (x[r,c] - mean_r) / sqrt(var_r + eps) * (scale_offset + gamma[g, c]) + beta[g, c]
+ * with g = r / rows_per_group, LayerNorm over the D features of row r, biased
+ * variance, fp32 statistics, no learned affine. scale_offset = 1 gives
+ * LN(x)(1+gamma)+beta; 0 gives the page's gamma*LN(x)+beta.
+ *   x, out      : [rows, D] bf16 (out may alias x)
+ *   gamma, beta : [rows / rows_per_group, D] bf16
+ * Errors: DIT_ERR_SHAPE unless rows >= 0, D > 0, D % 8 == 0, rows_per_group > 0,
+ * rows % rows_per_group == 0 and eps >= 0. rows == 0 is a no-op. */
+int dit_adaln_modulate(const void* x, const void* gamma, const void* beta, void* out,
+                       int64_t rows, int32_t D, int64_t rows_per_group, float eps,
+                       float scale_offset, void* stream);
+
+/* Gated residual (DiT page, "A ruptura da U-Net"): out = x + alpha_g * y, alpha
+ * a D-vector per group g = r / rows_per_group (a scalar gate is its broadcast;
+ * alpha = 0 returns x exactly, the adaLN-Zero identity).
+ *   x, y, out : [rows, D] bf16 (out may alias x or y);  alpha : [rows / rows_per_group, D] bf16
+ * Errors: as dit_adaln_modulate. */
+int dit_gated_residual(const void* x, const void* y, const void* alpha, void* out,
+                       int64_t rows, int32_t D, int64_t rows_per_group, void* stream);
+
+/* Standalone 3D-RoPE of q and k (DiT page, "3D-RoPE e atencao espaco-temporal"),
+ * fp32 rotation of bf16 data, the same rotation for every head.
+ *   q_in, k_in   : [rows, H, d] bf16; k_in may be NULL (then k_out is ignored)
+ *   q_out, k_out : [rows, H, d] bf16; may equal q_in / k_in (in place)
+ * Sequence layout: see the conventions above (positions restart per sequence).
+ * Errors: DIT_ERR_SHAPE unless d is 64 or 128, H > 0, the bands are even and sum
+ * to d, grid_h, grid_w >= 1, base > 1, offsets >= 0, and every sequence length
+ * is a multiple of grid_h * grid_w; DIT_ERR_SEQLENS for a bad cu_seqlens. */
+int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,
+                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                  const int32_t* cu_seqlens_host, const dit_rope3d_desc* rope, void* stream);
+
+/* Full non-causal attention per sequence and head (DiT page, "3D-RoPE e atencao
+ * espaco-temporal"; the Flowception summary: bidirectional attention over all
+ * frames), flash-style on tcgen05 tensor cores: bf16 operands, fp32 scores,
+ * fp32 online softmax and accumulation, bf16 output.
+ *   o[i, h, :] = sum_j softmax_j(scale * <q_rot[i,h], k_rot[j,h]>) v[j, h, :]
+ * over the keys j of the query's own sequence (packed sequences never see one
+ * another). With `rope` non-NULL, q and k are rotated by 3D-RoPE inside the
+ * kernel as their tiles are loaded (fp32 rotation, bf16 operand); with NULL they
+ * are used as given.
+ *   q, k, v, o : [rows, H, d] bf16, o must not overlap q, k or v
+ *   lse        : NULL or [rows, H] fp32, natural-log sum of exp(scale * scores)
+ *   softmax_scale <= 0 selects 1/sqrt(d).
+ * Errors: DIT_ERR_SHAPE unless d is 64 or 128, H > 0, rows > 0 ... (and, with
+ * rope, as dit_rope3d_qk); DIT_ERR_SEQLENS for a bad cu_seqlens; DIT_ERR_DEVICE
+ * off sm_100. */
+int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t rows,
+                 int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                 const int32_t* cu_seqlens_host, float softmax_scale, const dit_rope3d_desc* rope,
+                 void* stream);
+
+/* Waits for `stream`, then reads and clears the library's device error word.
+ * Returns DIT_ERR_TIMEOUT if any kernel gave up a bounded wait since the last
+ * check (its outputs are then invalid), DIT_ERR_LAUNCH on a CUDA error, else DIT_OK. */
+int dit_check_device(void* stream);
+
+/* Human-readable name of a dit_status code (static string, never NULL). */
+const char* dit_status_string(int status);
+
+/* Frees the cached RoPE tables of every device. Safe to call more than once. */
+void dit_shutdown(void);
+
+/* Test hook: 1 makes the next attention launches give up their first wait at once
+ * (exercising the bounded-wait error path without any hang), 0 restores. */
+void dit_debug_force_timeout(int enable);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT3D_H_ */

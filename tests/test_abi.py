@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/dit3d.h declares, and rejects bad arguments with the
+documented status codes before touching any device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from diffusion_transformer_video_b200 import build, dit3d
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return dit3d.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "dit3d.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dit_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("dit_adaln_modulate", "dit_rope3d_qk", "dit_attn_fwd", "dit_gated_residual"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert set(names) == set(dit3d.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code, name in dit3d.STATUS_NAMES.items():
+        assert L.dit_status_string(code).decode().startswith(name)
+    assert L.dit_status_string(99) == b"unknown dit_status"
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def test_validation_before_any_device_work(L):
+    # rows not a multiple of rows_per_group
+    assert L.dit_adaln_modulate(FAKE, FAKE, FAKE, FAKE, 10, 64, 3, 1e-6, 1.0, None) == 2
+    # D not a multiple of 8
+    assert L.dit_gated_residual(FAKE, FAKE, FAKE, FAKE, 4, 12, 4, None) == 2
+    # NULL pointer
+    assert L.dit_gated_residual(None, FAKE, FAKE, FAKE, 4, 16, 4, None) == 1
+    # misaligned pointer
+    assert L.dit_adaln_modulate(MISALIGNED, FAKE, FAKE, FAKE, 4, 64, 4, 1e-6, 1.0, None) == 3
+    # head_dim 96 unsupported
+    assert L.dit_attn_fwd(FAKE, FAKE, FAKE, FAKE, None, 10, 2, 96, 1, None, None, 0.0, None,
+                          None) == 2
+    # cu_seqlens on host only
+    cu = (ctypes.c_int32 * 3)(0, 5, 10)
+    assert L.dit_attn_fwd(FAKE, FAKE, FAKE, FAKE, None, 10, 2, 128, 2, None, cu, 0.0, None,
+                          None) == 1
+    # cu_seqlens not ending at rows / decreasing
+    bad = (ctypes.c_int32 * 3)(0, 5, 9)
+    assert L.dit_attn_fwd(FAKE, FAKE, FAKE, FAKE, None, 10, 2, 128, 2, FAKE, bad, 0.0, None,
+                          None) == 4
+    bad = (ctypes.c_int32 * 3)(0, 7, 5)
+    assert L.dit_rope3d_qk(FAKE, None, FAKE, None, 5, 2, 128, 2, FAKE, bad,
+                           ctypes.byref(dit3d.rope_desc(1, 1, (44, 42, 42))), None) == 4
+    # RoPE bands that do not sum to head_dim, odd band, sequence not a whole number of frames
+    assert L.dit_rope3d_qk(FAKE, None, FAKE, None, 16, 2, 128, 1, None, None,
+                           ctypes.byref(dit3d.rope_desc(2, 2, (44, 42, 40))), None) == 2
+    assert L.dit_rope3d_qk(FAKE, None, FAKE, None, 16, 2, 64, 1, None, None,
+                           ctypes.byref(dit3d.rope_desc(2, 2, (15, 25, 24))), None) == 2
+    assert L.dit_rope3d_qk(FAKE, None, FAKE, None, 18, 2, 64, 1, None, None,
+                           ctypes.byref(dit3d.rope_desc(2, 2, (16, 24, 24))), None) == 2
+
+
+@pytest.mark.skipif(os.environ.get("CUDA_VISIBLE_DEVICES", None) is None and
+                    not os.path.exists("/dev/nvidia0") is False, reason="GPU present")
+def test_valid_call_without_gpu_reports_device_error(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.dit_adaln_modulate(FAKE, FAKE, FAKE, FAKE, 4, 64, 4, 1e-6, 1.0, None) == 5

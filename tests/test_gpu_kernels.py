@@ -1,0 +1,234 @@
+"""GPU parity of every libdit3d call against the fp64 oracle on small and ragged
+cases (several tiles plus a ragged tail), edge cases and error paths. All calls
+go through the C ABI via the ctypes binding."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from diffusion_transformer_video_b200 import dit3d, workloads as wl
+from tests.helpers import check_attention, check_modulation, f64, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(7)
+
+
+def bits(shape, std=1.0):
+    return wl.f32_to_bf16_bits(RNG.standard_normal(shape).astype(np.float32) * np.float32(std))
+
+
+# ----------------------------------------------------------------------------- modulation
+
+@pytest.mark.parametrize("rows,D,rpg", [(1, 8, 1), (37, 128, 37), (64, 3072, 16), (20, 5120, 10),
+                                        (3, 1032, 1), (5, 9216, 5)])
+@pytest.mark.parametrize("s0", [1.0, 0.0])
+def test_adaln_modulate_parity(rows, D, rpg, s0):
+    x, g, b = bits((rows, D)), bits((rows // rpg, D), 0.1), bits((rows // rpg, D), 0.1)
+    out = dit3d.dit_adaln_modulate(to_dev(x), to_dev(g), to_dev(b), rpg, eps=1e-6, scale_offset=s0)
+    ref = oracle.adaln_modulate(f64(x), f64(g), f64(b), rpg, 1e-6, s0)
+    check_modulation(from_dev(out), ref, f"modulate rows={rows} D={D}")
+
+
+def test_adaln_modulate_in_place_and_constant_rows():
+    rows, D = 6, 256
+    x = np.repeat(wl.f32_to_bf16_bits(np.linspace(-3, 3, rows, dtype=np.float32))[:, None], D, 1)
+    g, b = bits((2, D), 0.1), bits((2, D), 0.1)
+    xt = to_dev(x)
+    dit3d.dit_adaln_modulate(xt, to_dev(g), to_dev(b), 3, out=xt)
+    # a constant row normalises to 0: the output is beta of the row's group, exactly
+    np.testing.assert_array_equal(from_dev(xt), np.repeat(f64(b), 3, axis=0))
+
+
+# ----------------------------------------------------------------------------- residual
+
+@pytest.mark.parametrize("rows,D,rpg", [(1, 8, 1), (64, 128, 64), (33, 3072, 11), (8, 5120, 2),
+                                        (2, 10240, 1)])
+def test_gated_residual_parity(rows, D, rpg):
+    x, y, a = bits((rows, D)), bits((rows, D)), bits((rows // rpg, D), 0.1)
+    out = dit3d.dit_gated_residual(to_dev(x), to_dev(y), to_dev(a), rpg)
+    ref = oracle.gated_residual(f64(x), f64(y), f64(a), rpg)
+    check_modulation(from_dev(out), ref, "residual")
+
+
+def test_gated_residual_alpha_zero_is_bitwise_identity():
+    x, y = bits((50, 3072)), bits((50, 3072), 30.0)
+    xt = to_dev(x)
+    out = dit3d.dit_gated_residual(xt, to_dev(y), torch.zeros(2, 3072, dtype=torch.bfloat16,
+                                                              device="cuda"), 25)
+    assert torch.equal(out.view(torch.int16), xt.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- RoPE
+
+def _rope_ref(v_bits, cu, grid_h, grid_w, bands, base=10000.0, offsets=(0, 0, 0)):
+    return oracle.rope3d(f64(v_bits), cu, grid_h, grid_w, bands, base, offsets)
+
+
+@pytest.mark.parametrize("d,bands,gh,gw,frames", [(64, (16, 24, 24), 4, 4, [4]),
+                                                   (128, (44, 42, 42), 3, 5, [2, 7, 1]),
+                                                   (128, (32, 48, 48), 8, 8, [1, 1])])
+def test_rope3d_parity(d, bands, gh, gw, frames):
+    H = 3
+    lens = [f * gh * gw for f in frames]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    rows = int(cu[-1])
+    q, k = bits((rows, H, d)), bits((rows, H, d))
+    desc = dit3d.rope_desc(gh, gw, bands, 10000.0, (1, 2, 3))
+    qo, ko = dit3d.dit_rope3d_qk(to_dev(q), to_dev(k), desc, cu_seqlens=cu)
+    for got, src in ((qo, q), (ko, k)):
+        ref = _rope_ref(src, cu, gh, gw, bands, 10000.0, (1, 2, 3))
+        err = np.abs(from_dev(got) - ref)
+        # fp32 rotation then one bf16 rounding: within a bf16 half-ulp (+ fp32 slack)
+        from tests.helpers import half_ulp_bf16
+        assert (err <= half_ulp_bf16(ref) * 1.01 + 1e-6).all(), err.max()
+
+
+def test_rope3d_dense_in_place_equals_out_of_place():
+    gh, gw, T, H, d = 6, 7, 3, 4, 128
+    rows = 2 * T * gh * gw
+    q, k = bits((rows, H, d)), bits((rows, H, d))
+    desc = dit3d.rope_desc(gh, gw, (44, 42, 42))
+    qa, ka = dit3d.dit_rope3d_qk(to_dev(q), to_dev(k), desc, n_seq=2)
+    qt, kt = to_dev(q), to_dev(k)
+    dit3d.dit_rope3d_qk(qt, kt, desc, n_seq=2, inplace=True)
+    assert torch.equal(qa, qt) and torch.equal(ka, kt)
+    # dense with two sequences == packed layout with the same boundaries
+    qp, _ = dit3d.dit_rope3d_qk(to_dev(q), None, desc, cu_seqlens=[0, rows // 2, rows])
+    assert torch.equal(qp, qa)
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _attn_case(lens, H, d, rope=None, q_scale=1.0, same_qk=False, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = int(sum(lens))
+    mk = lambda s=1.0: wl.f32_to_bf16_bits(rng.standard_normal((rows, H, d)).astype(np.float32) * np.float32(s))
+    q, k, v = mk(q_scale), mk(), mk()
+    if same_qk:
+        k = q.copy()
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return q, k, v, cu
+
+
+def _run_attn(q, k, v, cu, rope_kw=None, varlen=True, n_seq=1):
+    desc = dit3d.rope_desc(**rope_kw) if rope_kw else None
+    o, lse = dit3d.dit_attn_fwd(to_dev(q), to_dev(k), to_dev(v), n_seq=n_seq,
+                                cu_seqlens=cu if varlen else None, rope=desc, return_lse=True)
+    dit3d.dit_check_device()
+    return from_dev(o), lse.cpu().double().numpy()
+
+
+@pytest.mark.parametrize("lens,H,d", [([64], 2, 64), ([128], 1, 128), ([300], 2, 128),
+                                      ([256], 2, 64), ([1], 1, 128), ([513], 1, 128)])
+def test_attn_dense_parity(lens, H, d):
+    q, k, v, cu = _attn_case(lens, H, d)
+    o, lse = _run_attn(q, k, v, cu, varlen=False)
+    ref_o, ref_lse = oracle.attn_fwd(f64(q), f64(k), f64(v), cu)
+    check_attention(o, ref_o, f"attn {lens}")
+    np.testing.assert_allclose(lse, ref_lse, atol=2e-2)
+
+
+def test_attn_dense_batch_equals_packed():
+    q, k, v, cu = _attn_case([200, 200, 200], 2, 128)
+    o_dense, _ = _run_attn(q, k, v, cu, varlen=False, n_seq=3)
+    o_pack, _ = _run_attn(q, k, v, cu, varlen=True)
+    np.testing.assert_array_equal(o_dense, o_pack)
+    ref, _ = oracle.attn_fwd(f64(q), f64(k), f64(v), cu)
+    check_attention(o_dense, ref, "batch")
+
+
+@pytest.mark.parametrize("lens", [[130, 1, 255, 16, 400], [128, 256], [7, 0, 90]])
+def test_attn_varlen_parity(lens):
+    q, k, v, cu = _attn_case(lens, 2, 128, seed=3)
+    o, lse = _run_attn(q, k, v, cu)
+    ref_o, ref_lse = oracle.attn_fwd(f64(q), f64(k), f64(v), cu)
+    check_attention(o, ref_o, f"varlen {lens}")
+    np.testing.assert_allclose(lse, ref_lse, atol=2e-2)
+
+
+@pytest.mark.parametrize("d,bands,gh,gw,frames", [(64, (16, 24, 24), 4, 4, [4]),
+                                                   (128, (44, 42, 42), 3, 5, [9, 2, 20]),
+                                                   (128, (32, 48, 48), 16, 16, [1])])
+def test_attn_fused_rope_parity(d, bands, gh, gw, frames):
+    lens = [f * gh * gw for f in frames]
+    q, k, v, cu = _attn_case(lens, 2, d, seed=11)
+    rope_kw = dict(grid_h=gh, grid_w=gw, bands=bands, base=10000.0, offsets=(0, 1, 2))
+    o, lse = _run_attn(q, k, v, cu, rope_kw)
+    ref_o, ref_lse = oracle.attn_fwd(f64(q), f64(k), f64(v), cu, rope=rope_kw)
+    check_attention(o, ref_o, "fused rope")
+    np.testing.assert_allclose(lse, ref_lse, atol=2e-2)
+
+
+def test_attn_fused_rope_equals_rope_then_attn():
+    gh, gw, frames = 5, 6, [7, 3]
+    lens = [f * gh * gw for f in frames]
+    q, k, v, cu = _attn_case(lens, 3, 128, seed=5)
+    desc = dit3d.rope_desc(gh, gw, (44, 42, 42))
+    qr, kr = dit3d.dit_rope3d_qk(to_dev(q), to_dev(k), desc, cu_seqlens=cu)
+    o_two = dit3d.dit_attn_fwd(qr, kr, to_dev(v), cu_seqlens=cu)
+    o_fused = dit3d.dit_attn_fwd(to_dev(q), to_dev(k), to_dev(v), cu_seqlens=cu, rope=desc)
+    # both round the rotated operands to bf16 with the same fp32 rotation: identical
+    assert torch.equal(o_two, o_fused)
+
+
+@pytest.mark.parametrize("case", ["sharp_q", "q_equals_k"])
+def test_attn_sharpened_softmax(case):
+    # unit-normal scores are nearly uniform; sharpen them to exercise the online rescale
+    q, k, v, cu = _attn_case([700], 2, 128, q_scale=4.0 if case == "sharp_q" else 1.0,
+                             same_qk=(case == "q_equals_k"), seed=9)
+    o, lse = _run_attn(q, k, v, cu)
+    ref_o, ref_lse = oracle.attn_fwd(f64(q), f64(k), f64(v), cu)
+    check_attention(o, ref_o, case)
+    np.testing.assert_allclose(lse, ref_lse, atol=5e-2)
+
+
+def test_attn_softmax_scale_and_invariants():
+    q, k, _, cu = _attn_case([333], 2, 64, seed=2)
+    ones = np.full((333, 2, 64), 0x3F80, np.uint16)  # bf16(1.0)
+    o, _ = _run_attn(q, k, ones, cu)
+    np.testing.assert_allclose(o, 1.0, atol=4e-3)  # rows of P sum to one
+    vrand = wl.f32_to_bf16_bits(RNG.standard_normal((333, 2, 64)).astype(np.float32))
+    o2 = dit3d.dit_attn_fwd(to_dev(q), to_dev(k), to_dev(vrand), softmax_scale=0.05)
+    ref, _ = oracle.attn_fwd(f64(q), f64(k), f64(vrand), cu, scale=0.05)
+    check_attention(from_dev(o2), ref, "scale")
+
+
+# ----------------------------------------------------------------------------- errors
+
+def test_validation_errors_return_status():
+    x = torch.zeros(4, 16, dtype=torch.bfloat16, device="cuda")
+    g = torch.zeros(1, 16, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_adaln_modulate(x, g, g, rows_per_group=3)
+    assert e.value.status == 2
+    q = torch.zeros(10, 1, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_attn_fwd(q, q, q)
+    assert e.value.status == 2
+    q = torch.zeros(10, 1, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_attn_fwd(q, q, q, cu_seqlens=[0, 6, 5, 10])
+    assert e.value.status == 4
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_attn_fwd(q, q, q, rope=dit3d.rope_desc(2, 2, (44, 42, 40)))
+    assert e.value.status == 2
+    raw = dit3d.lib().dit_attn_fwd(None, None, None, None, None, 10, 1, 128, 1, None, None, 0.0,
+                                   None, None)
+    assert raw == 1
+
+
+def test_bounded_wait_reports_timeout_without_hanging():
+    q = torch.randn(300, 2, 128, device="cuda").to(torch.bfloat16)
+    dit3d.lib().dit_debug_force_timeout(1)
+    try:
+        dit3d.dit_attn_fwd(q, q, q)
+        with pytest.raises(dit3d.DitError) as e:
+            dit3d.dit_check_device()
+        assert e.value.status == 7
+    finally:
+        dit3d.lib().dit_debug_force_timeout(0)
+    # the context is still usable and the error word was cleared
+    o = dit3d.dit_attn_fwd(q, q, q)
+    dit3d.dit_check_device()
+    assert torch.isfinite(o.float()).all()
