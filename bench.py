@@ -160,6 +160,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=24, help="oracle sample rows per step")
     ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (smaller cases for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -186,6 +188,9 @@ def main():
             dist.barrier()
 
     w = wl.get_workload(args.workload, args.seed)
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}-h{args.heads}", heads=args.heads)
     # every rank runs its own batch of the workload (seeded per rank)
     seed = args.seed + 1000 * rank
     inp = wl.make_inputs(w, seed)
@@ -254,14 +259,15 @@ def main():
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.e2e_steps):
+    n_e2e = max(args.e2e_steps, 1)
+    for _ in range(n_e2e):
         for k in e2e_keys:
             dev2[k].copy_(host[k], non_blocking=True)
         step(dev2)
         res_host.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
 
     flops = w.attn_flops()
     ms_step = elapsed_ms / K
