@@ -148,6 +148,26 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Every rank draws its own batch of the workload."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Elementwise max of per-rank timings (the slowest rank sets the job's time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: the units all ranks processed / the max-over-ranks step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -160,6 +180,10 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=24, help="oracle sample rows per step")
     ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rope-mode", default="fused", choices=["fused", "prepass", "none"],
+                    help="fused: RoPE inside the attention kernel (the product path); prepass: "
+                         "dit_rope3d_qk into scratch then attention; none: attention alone "
+                         "(not the workload, a kernel-speed reference)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (smaller cases for profiling)")
     args = ap.parse_args()
@@ -192,7 +216,7 @@ def main():
         import dataclasses
         w = dataclasses.replace(w, name=f"{w.name}-h{args.heads}", heads=args.heads)
     # every rank runs its own batch of the workload (seeded per rank)
-    seed = args.seed + 1000 * rank
+    seed = rank_seed(args.seed, rank)
     inp = wl.make_inputs(w, seed)
     host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
             for k, v in inp.items()}
@@ -209,14 +233,27 @@ def main():
     out = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
 
+    if args.rope_mode == "prepass":
+        q_rot, k_rot = torch.empty_like(dev["q"]), torch.empty_like(dev["k"])
+
+    def attention(b):
+        if args.rope_mode == "fused":
+            dit3d.dit_attn_fwd(b["q"], b["k"], b["v"], n_seq=w.n_seq, cu_seqlens=cu, rope=desc,
+                               out=o)
+        elif args.rope_mode == "prepass":
+            dit3d.dit_rope3d_qk(b["q"], b["k"], desc, n_seq=w.n_seq, cu_seqlens=cu,
+                                q_out=q_rot, k_out=k_rot)
+            dit3d.dit_attn_fwd(q_rot, k_rot, b["v"], n_seq=w.n_seq, cu_seqlens=cu, out=o)
+        else:
+            dit3d.dit_attn_fwd(b["q"], b["k"], b["v"], n_seq=w.n_seq, cu_seqlens=cu, out=o)
+
     def step(b, ev=None):
         if ev is not None:
             ev[0].record(stream)
         dit3d.dit_adaln_modulate(b["x"], b["gamma"], b["beta"], rpg, out=u)
         if ev is not None:
             ev[1].record(stream)
-        dit3d.dit_attn_fwd(b["q"], b["k"], b["v"], n_seq=w.n_seq, cu_seqlens=cu, rope=desc,
-                           out=o)
+        attention(b)
         if ev is not None:
             ev[2].record(stream)
         dit3d.dit_gated_residual(b["x"], o.view(rows, D), b["alpha"], rpg, out=out)
@@ -271,12 +308,9 @@ def main():
 
     flops = w.attn_flops()
     ms_step = elapsed_ms / K
-    if world > 1:
-        tt = torch.tensor([ms_step, e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step, e2e_ms = float(tt[0]), float(tt[1])
-    value = flops * world / (ms_step * 1e-3) / 1e12
-    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+    ms_step, e2e_ms = max_over_ranks([ms_step, e2e_ms], dist if world > 1 else None, "cuda")
+    value = job_throughput(flops, world, ms_step)
+    e2e_value = job_throughput(flops, world, e2e_ms)
 
     pk = _peaks()
     att_tflops = flops / (t_att * 1e-3) / 1e12
@@ -304,12 +338,14 @@ def main():
                        "l2": "inputs larger than L2 (x, q, k, v are %.0f MB each)" % (rows * D * 2 / 1e6)
                        if rows * D * 2 > 126e6 else "inputs smaller than L2 (no flush)",
                        "note": w.note},
-            "gpu_launches": 3 * K,
+            "gpu_launches": (4 if args.rope_mode == "prepass" else 3) * K,
             "roofline": {"bound": "tensor", "achieved": att_tflops,
                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": att_tflops / pk["bf16_tflops_sustained"],
                          "traffic": ATTN_DRAM_BYTES_PER_LAUNCH,
-                         "kernel": "dit_attn_fwd (fused 3D-RoPE)",
+                         "kernel": {"fused": "dit_attn_fwd (fused 3D-RoPE)",
+                                    "prepass": "dit_rope3d_qk + dit_attn_fwd",
+                                    "none": "dit_attn_fwd without RoPE"}[args.rope_mode],
                          "peak_source": f"{pk['source']} sustained bf16 "
                                         f"(burst {pk['bf16_tflops']}: frac "
                                         f"{att_tflops / pk['bf16_tflops']:.3f})"},

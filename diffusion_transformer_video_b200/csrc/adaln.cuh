@@ -134,6 +134,17 @@ adaln_modulate_wide_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restri
   }
 }
 
+// x + a*y on a bf16 pair. A zero gate returns x's bits unchanged (the adaLN-Zero
+// identity holds exactly, -0.0 included, whatever y holds).
+__device__ __forceinline__ float gate1(float x, float y, float a) {
+  return a == 0.f ? x : fmaf(a, y, x);
+}
+__device__ __forceinline__ uint32_t gate_pair(uint32_t xw, uint32_t yw, uint32_t aw) {
+  // bf16 -> fp32 -> bf16 of an unchanged x is exact, so a zero gate keeps x's bits
+  return pack_bf16x2(gate1(bf16lo(xw), bf16lo(yw), bf16lo(aw)),
+                     gate1(bf16hi(xw), bf16hi(yw), bf16hi(aw)));
+}
+
 template <int NV>
 __global__ void __launch_bounds__(kRowThreads)
 gated_residual_kernel(const __nv_bfloat16* x, const __nv_bfloat16* y,
@@ -165,9 +176,7 @@ gated_residual_kernel(const __nv_bfloat16* x, const __nv_bfloat16* y,
       const uint32_t aw[4] = {av[k].x, av[k].y, av[k].z, av[k].w};
       uint32_t o[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        o[e] = pack_bf16x2(fmaf(bf16lo(aw[e]), bf16lo(yw[e]), bf16lo(xw[e])),
-                           fmaf(bf16hi(aw[e]), bf16hi(yw[e]), bf16hi(xw[e])));
+      for (int e = 0; e < 4; ++e) o[e] = gate_pair(xw[e], yw[e], aw[e]);
       st_stream(orow + c * 16, make_uint4(o[0], o[1], o[2], o[3]));
     }
   }
@@ -188,9 +197,7 @@ gated_residual_wide_kernel(const __nv_bfloat16* x, const __nv_bfloat16* y,
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, yw[4] = {yv.x, yv.y, yv.z, yv.w},
                    aw[4] = {av.x, av.y, av.z, av.w};
     uint32_t o[4];
-    for (int e = 0; e < 4; ++e)
-      o[e] = pack_bf16x2(fmaf(bf16lo(aw[e]), bf16lo(yw[e]), bf16lo(xw[e])),
-                         fmaf(bf16hi(aw[e]), bf16hi(yw[e]), bf16hi(xw[e])));
+    for (int e = 0; e < 4; ++e) o[e] = gate_pair(xw[e], yw[e], aw[e]);
     st_stream(reinterpret_cast<char*>(out) + off + c * 16, make_uint4(o[0], o[1], o[2], o[3]));
   }
 }

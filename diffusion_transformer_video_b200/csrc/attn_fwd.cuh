@@ -8,14 +8,20 @@
 // it lives in tensor memory one 128 x 128 tile at a time.)
 //
 // One CTA computes two 128-row query tiles (Q0, Q1) of one head of one sequence
-// and streams the sequence's keys/values in 128-row tiles through a 2-stage
-// shared-memory ring. 384 threads in three warpgroups:
+// and streams the sequence's keys/values in 128-row tiles through shared-memory
+// rings. 512 threads in four warpgroups:
 //   WG0 (warps 0-3)  softmax of Q0: thread i owns query row i = TMEM lane i.
 //   WG1 (warps 4-7)  softmax of Q1.
-//   warp 8           TMA producer: Q0, Q1 once, then K_j, V_j per stage.
-//   warp 9           TMEM allocator and tcgen05.mma issuer (one thread).
-//   warps 10-11      3D-RoPE: rotate Q0/Q1 and every K_j in shared memory, in
+//   WG2 (warps 8-11) 3D-RoPE: rotate Q0/Q1 and every K_j in shared memory, in
 //                    place, right after TMA lands them (fp32 math, bf16 result).
+//   warp 12          TMA producer of Q0, Q1 (once) and of the 3-stage K ring.
+//   warp 13          TMEM allocator and tcgen05.mma issuer (one thread).
+//   warp 14          TMA producer of the 2-stage V ring.
+//   warp 15          idle (it only gives its registers away).
+// A K stage is released right after both QK^T products read it, a V stage after
+// both PV products, so K tiles (and their RoPE) run up to three tiles ahead.
+// setmaxnreg moves registers to the softmax warpgroups (184 each; 80 for RoPE, 64 else)
+// so a thread can hold its whole 128-column score row.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
 // O1 [384,384+d). P_i (bf16, two per column) overwrites the first 64 columns of
 // S_i once the softmax has read S_i into registers.
@@ -38,12 +44,15 @@
 namespace dit3d {
 namespace attn {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
-constexpr int kStages = 2;
-constexpr int kRopeThreads = 64;
-constexpr int kWarpTma = 8, kWarpMma = 9, kWarpRope0 = 10;
+constexpr int kKStages = 3;  // K ring: released as soon as both Q tiles' QK^T read it
+constexpr int kVStages = 2;  // V ring: released after both PV products
+constexpr int kRopeThreads = 128;
+constexpr int kWarpRope0 = 8, kWarpTma = 12, kWarpMma = 13, kWarpTmaV = 14;
+// register split (setmaxnreg): 2*128*184 + 128*80 + 128*64 = 65536 = 512*128
+constexpr int kSoftmaxRegs = 184, kRopeRegs = 80, kCtrlRegs = 64;
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int qi) { return qi ? 128u : 0u; }
 __host__ __device__ constexpr uint32_t col_o(int qi) { return qi ? 384u : 256u; }
@@ -68,15 +77,16 @@ struct Smem {
   static constexpr uint32_t kTile = kTileM * D * 2;           // one Q, K or V tile
   static constexpr uint32_t kQ0 = 0, kQ1 = kTile;
   static constexpr uint32_t kK = 2 * kTile;                   // + stage * kTile
-  static constexpr uint32_t kV = kK + kStages * kTile;        // + stage * kTile
-  static constexpr uint32_t kBytes = kV + kStages * kTile;
+  static constexpr uint32_t kV = kK + kKStages * kTile;       // + stage * kTile
+  static constexpr uint32_t kBytes = kV + kVStages * kTile;
   // dynamic smem request: forces one CTA per SM (the CTA takes all 512 TMEM columns)
   static constexpr uint32_t kRequest = (kBytes + 1024 > 120 * 1024) ? kBytes + 1024 : 120 * 1024;
 };
 
 struct Barriers {
   uint64_t q_full, q_ready;
-  uint64_t k_full[kStages], v_full[kStages], k_ready[kStages], kv_empty[kStages];
+  uint64_t k_full[kKStages], k_ready[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_final, drain;
 };
@@ -94,31 +104,46 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int cc) {
 }
 
 // Rotate rows [0, n_valid) of one tile in shared memory. Row r of the tile is
-// token (row0 + r) of its sequence. Runs on the kRopeThreads RoPE threads.
+// token (row0 + r) of its sequence. Runs on the kRopeThreads RoPE threads; each
+// thread owns one 16-byte column chunk and walks rows two at a time so the
+// table lookups of four rows are in flight together.
 template <int D>
 __device__ __forceinline__ void rope_tile(uint8_t* tile, int64_t row0, int n_valid,
                                           const RopeParams& rp, int rt, int* s_pos) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RPP = kRopeThreads / CPR;    // rows per pass
-  // positions of the tile rows, packed t | h << 11 | w << 22 (host checks the ranges)
-  for (int r = rt; r < kTileM; r += kRopeThreads) {
+  static_assert(kRopeThreads == kTileM, "one position per thread");
+  {
+    // position of tile row rt, packed t | h << 11 | w << 22 (host checks the ranges)
     int t = 0, h = 0, w = 0;
-    if (r < n_valid) token_pos(row0 + r, rp.grid_h, rp.grid_w, t, h, w);
-    s_pos[r] = t | (h << 11) | (w << 22);
+    if (rt < n_valid) token_pos(row0 + rt, rp.grid_h, rp.grid_w, t, h, w);
+    s_pos[rt] = t | (h << 11) | (w << 22);
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");
   const int cc = rt % CPR;
   PairRef pr[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) pr[e] = rope_pair_ref(rp, cc * 4 + e);
-  for (int r = rt / CPR; r < n_valid; r += RPP) {
-    const int pk = s_pos[r];
-    const int t = pk & 2047, h = (pk >> 11) & 2047, w = (pk >> 22) & 1023;
-    uint4* p = reinterpret_cast<uint4*>(tile + sw128_chunk(r, cc));
-    float2 cs[4];
+  for (int base = rt / CPR; base < n_valid; base += 2 * RPP) {
+    uint4 v[2];
+    float2 cs[2][4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) cs[e] = rope_cs(rp, pr[e], t, h, w);
-    *p = rope_rotate_chunk(*p, cs);
+    for (int u = 0; u < 2; ++u) {
+      const int r = base + u * RPP;
+      if (r < n_valid) {
+        const int pk = s_pos[r];
+        const int t = pk & 2047, h = (pk >> 11) & 2047, w = (pk >> 22) & 1023;
+        v[u] = *reinterpret_cast<const uint4*>(tile + sw128_chunk(r, cc));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cs[u][e] = rope_cs(rp, pr[e], t, h, w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = base + u * RPP;
+      if (r < n_valid)
+        *reinterpret_cast<uint4*>(tile + sw128_chunk(r, cc)) = rope_rotate_chunk(v[u], cs[u]);
+    }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");  // s_pos reuse
 }
@@ -175,11 +200,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     s_abort = p.force_timeout ? 1 : 0;
     ptx::mbar_init(ptx::smem_u32(&b->q_full), 1);
     ptx::mbar_init(ptx::smem_u32(&b->q_ready), kRopeThreads);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       ptx::mbar_init(ptx::smem_u32(&b->k_full[s]), 1);
-      ptx::mbar_init(ptx::smem_u32(&b->v_full[s]), 1);
       ptx::mbar_init(ptx::smem_u32(&b->k_ready[s]), kRopeThreads);
-      ptx::mbar_init(ptx::smem_u32(&b->kv_empty[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&b->k_empty[s]), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&b->v_full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&b->v_empty[s]), 1);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(ptx::smem_u32(&b->s_full[i]), 1);
@@ -197,6 +225,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = s_tmem_base;
+
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+  } else if (warp < 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRopeRegs));
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+  }
 
   if (warp < 8) {
     // =========================================================== softmax warpgroups
@@ -218,7 +254,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
       for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + c * 32, sr + c * 32);
       ptx::tmem_wait_ld();
-      float* s = reinterpret_cast<float*>(sr);
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
       if (j == nk - 1 && last_valid < kTileN) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -238,31 +276,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // warp-collective O rescale (lanes that keep their max use factor 1)
         const float f = raise ? ex2(m - mcand) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(tO + c * 32, ov);
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t ov[16];
+          ptx::tmem_ld16(tO + c * 16, ov);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
-          ptx::tmem_st32(tO + c * 32, ov);
+          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
+          ptx::tmem_st16(tO + c * 16, ov);
         }
         l *= f;
       }
       if (raise) m = mcand;
       const float neg_m = -m;
       float l0 = 0.f, l1 = 0.f;
-      uint32_t pw[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float e0 = ex2(fmaf(s[2 * c], p.scale_log2, neg_m));
-        const float e1 = ex2(fmaf(s[2 * c + 1], p.scale_log2, neg_m));
-        l0 += e0;
-        l1 += e1;
-        pw[c] = pack_bf16x2(e0, e1);
+      for (int q4 = 0; q4 < 4; ++q4) {
+        // P for 32 keys -> 16 packed columns, stored as soon as they are ready
+        uint32_t pw[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float e0 = ex2(fmaf(s[32 * q4 + 2 * c], p.scale_log2, neg_m));
+          const float e1 = ex2(fmaf(s[32 * q4 + 2 * c + 1], p.scale_log2, neg_m));
+          l0 += e0;
+          l1 += e1;
+          pw[c] = pack_bf16x2(e0, e1);
+        }
+        ptx::tmem_st16(tS + 16 * q4, pw);
       }
       l += l0 + l1;
-      ptx::tmem_st32(tS, pw);
-      ptx::tmem_st32(tS + 32, pw + 32);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar_p);
@@ -295,48 +336,49 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (valid && p.lse != nullptr)
         p.lse[(seq_start + row_in_seq) * p.H + head] = (m + __log2f(l)) * 0.69314718055994531f;
     }
-  } else if (warp == kWarpTma) {
-    // =========================================================== TMA producer
+  } else if (warp == kWarpTma || warp == kWarpTmaV) {
+    // =========================================================== TMA producers
+    // warp 12 loads Q once and then the K ring; warp 14 loads the V ring.
     if (lane == 0) {
-      ptx::prefetch_tmap(&tm_q);
-      ptx::prefetch_tmap(&tm_k);
-      ptx::prefetch_tmap(&tm_v);
+      const bool is_k = warp == kWarpTma;
+      const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+      const int stages = is_k ? kKStages : kVStages;
+      const uint32_t ring = is_k ? L::kK : L::kV;
+      uint64_t* full = is_k ? b->k_full : b->v_full;
+      uint64_t* empty = is_k ? b->k_empty : b->v_empty;
+      ptx::prefetch_tmap(tm);
       const int x0 = head * D;
       const uint32_t q_full = ptx::smem_u32(&b->q_full);
-      int issued = 0;  // K/V tiles issued
+      int issued = 0;  // tiles issued into this ring
       if (!*abort) {
-        ptx::mbar_arrive_expect_tx(q_full, 2 * L::kTile);
-        for (int qi = 0; qi < 2; ++qi)
-          for (int blk = 0; blk < D / 64; ++blk)
-            ptx::tma_load_2d(ptx::smem_u32(smem + (qi ? L::kQ1 : L::kQ0) + blk * 16384), &tm_q,
-                             x0 + blk * 64, static_cast<int>(seq_start + q_row0 + qi * kTileM),
-                             q_full);
+        if (is_k) {
+          ptx::prefetch_tmap(&tm_q);
+          ptx::mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+          for (int qi = 0; qi < 2; ++qi)
+            for (int blk = 0; blk < D / 64; ++blk)
+              ptx::tma_load_2d(ptx::smem_u32(smem + (qi ? L::kQ1 : L::kQ0) + blk * 16384), &tm_q,
+                               x0 + blk * 64, static_cast<int>(seq_start + q_row0 + qi * kTileM),
+                               q_full);
+        }
         for (int j = 0; j < nk; ++j) {
-          const int st = j % kStages;
-          if (j >= kStages &&
-              !ptx::mbar_wait(ptx::smem_u32(&b->kv_empty[st]), ((j / kStages) - 1) & 1, abort))
+          const int st = j % stages;
+          if (j >= stages &&
+              !ptx::mbar_wait(ptx::smem_u32(&empty[st]), ((j / stages) - 1) & 1, abort))
             break;
           const int y = static_cast<int>(seq_start + static_cast<int64_t>(j) * kTileN);
-          const uint32_t kf = ptx::smem_u32(&b->k_full[st]), vf = ptx::smem_u32(&b->v_full[st]);
-          ptx::mbar_arrive_expect_tx(kf, L::kTile);
+          const uint32_t f = ptx::smem_u32(&full[st]);
+          ptx::mbar_arrive_expect_tx(f, L::kTile);
           for (int blk = 0; blk < D / 64; ++blk)
-            ptx::tma_load_2d(ptx::smem_u32(smem + L::kK + st * L::kTile + blk * 16384), &tm_k,
-                             x0 + blk * 64, y, kf);
-          ptx::mbar_arrive_expect_tx(vf, L::kTile);
-          for (int blk = 0; blk < D / 64; ++blk)
-            ptx::tma_load_2d(ptx::smem_u32(smem + L::kV + st * L::kTile + blk * 16384), &tm_v,
-                             x0 + blk * 64, y, vf);
+            ptx::tma_load_2d(ptx::smem_u32(smem + ring + st * L::kTile + blk * 16384), tm,
+                             x0 + blk * 64, y, f);
           ++issued;
         }
         // drain: no copy may still be in flight into shared memory when the CTA exits
         // (normally these phases completed long ago and the waits return at once)
         volatile int never = 0;
-        ptx::mbar_wait(q_full, 0, &never);
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
-          const int st = j % kStages;
-          ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), (j / kStages) & 1, &never);
-          ptx::mbar_wait(ptx::smem_u32(&b->v_full[st]), (j / kStages) & 1, &never);
-        }
+        if (is_k) ptx::mbar_wait(q_full, 0, &never);
+        for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+          ptx::mbar_wait(ptx::smem_u32(&full[j % stages]), (j / stages) & 1, &never);
       }
     }
     __syncwarp();
@@ -374,28 +416,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_after();
         qk(0, 0);
         qk(1, 0);
+        ptx::umma_commit(ptx::smem_u32(&b->k_empty[0]));
         issued_any = true;
       }
       for (int j = 0; ok && j < nk; ++j) {
-        const int st = j % kStages, ph = (j / kStages) & 1;
-        const int st1 = (j + 1) % kStages, ph1 = ((j + 1) / kStages) & 1;
+        const int vs = j % kVStages, vph = (j / kVStages) & 1;
+        const int ks1 = (j + 1) % kKStages, kph1 = ((j + 1) / kKStages) & 1;
         const bool more = j + 1 < nk;
-        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[st]), ph, abort))) break;
+        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[vs]), vph, abort))) break;
         if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->p_full[0]), j & 1, abort))) break;
         ptx::tc_fence_after();
-        pv(0, st, j > 0);
+        pv(0, vs, j > 0);
         if (more) {
           if (!(ok = ptx::mbar_wait(
-                    ptx::smem_u32(p.use_rope ? &b->k_ready[st1] : &b->k_full[st1]), ph1, abort)))
+                    ptx::smem_u32(p.use_rope ? &b->k_ready[ks1] : &b->k_full[ks1]), kph1, abort)))
             break;
           ptx::tc_fence_after();
-          qk(0, st1);
+          qk(0, ks1);
         }
         if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->p_full[1]), j & 1, abort))) break;
         ptx::tc_fence_after();
-        pv(1, st, j > 0);
-        ptx::umma_commit(ptx::smem_u32(&b->kv_empty[st]));
-        if (more) qk(1, st1);
+        pv(1, vs, j > 0);
+        ptx::umma_commit(ptx::smem_u32(&b->v_empty[vs]));
+        if (more) {
+          qk(1, ks1);
+          ptx::umma_commit(ptx::smem_u32(&b->k_empty[ks1]));
+        }
       }
       if (ok) ptx::umma_commit(ptx::smem_u32(&b->o_final));
       if (issued_any) {
@@ -406,7 +452,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp >= kWarpRope0 && warp < kWarpRope0 + 4) {
     // =========================================================== 3D-RoPE warps
     if (p.use_rope) {
       const int rt = tid - kWarpRope0 * 32;
@@ -432,7 +478,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
         for (int j = 0; j < nk; ++j) {
-          const int st = j % kStages, ph = (j / kStages) & 1;
+          const int st = j % kKStages, ph = (j / kKStages) & 1;
           if (!all_ok(ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort))) break;
           const int nv = (j == nk - 1) ? last_valid : kTileN;
           rope_tile<D>(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv, p.rope,
