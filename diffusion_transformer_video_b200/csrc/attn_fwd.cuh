@@ -14,12 +14,13 @@
 //   WG1 (warps 4-7)  softmax of Q1.
 //   WG2 (warps 8-11) 3D-RoPE: rotate Q0/Q1 and every K_j in shared memory, in
 //                    place, right after TMA lands them (fp32 math, bf16 result).
-//   warp 12          TMA producer of Q0, Q1 (once) and of the 3-stage K ring.
+//   warp 12          TMA producer of Q0, Q1 (once) and of the 2-stage K ring.
 //   warp 13          TMEM allocator and tcgen05.mma issuer (one thread).
 //   warp 14          TMA producer of the 2-stage V ring.
 //   warp 15          idle (it only gives its registers away).
 // A K stage is released right after both QK^T products read it, a V stage after
-// both PV products, so K tiles (and their RoPE) run up to three tiles ahead.
+// both PV products, so K tiles (and their RoPE) run ahead of the V tiles. The
+// RoPE cos/sin table (up to 32 KB) is copied into shared memory once per CTA.
 // setmaxnreg moves registers to the softmax warpgroups (184 each; 80 for RoPE, 64 else)
 // so a thread can hold its whole 128-column score row.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
@@ -47,7 +48,7 @@ namespace attn {
 constexpr int kThreads = 512;
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;
-constexpr int kKStages = 3;  // K ring: released as soon as both Q tiles' QK^T read it
+constexpr int kKStages = 2;  // K ring: released as soon as both Q tiles' QK^T read it
 constexpr int kVStages = 2;  // V ring: released after both PV products
 constexpr int kRopeThreads = 128;
 constexpr int kWarpRope0 = 8, kWarpTma = 12, kWarpMma = 13, kWarpTmaV = 14;
@@ -78,7 +79,9 @@ struct Smem {
   static constexpr uint32_t kQ0 = 0, kQ1 = kTile;
   static constexpr uint32_t kK = 2 * kTile;                   // + stage * kTile
   static constexpr uint32_t kV = kK + kKStages * kTile;       // + stage * kTile
-  static constexpr uint32_t kBytes = kV + kVStages * kTile;
+  static constexpr uint32_t kTab = kV + kVStages * kTile;     // RoPE cos/sin table copy
+  static constexpr uint32_t kTabBytes = 32 * 1024;
+  static constexpr uint32_t kBytes = kTab + kTabBytes;
   // dynamic smem request: forces one CTA per SM (the CTA takes all 512 TMEM columns)
   static constexpr uint32_t kRequest = (kBytes + 1024 > 120 * 1024) ? kBytes + 1024 : 120 * 1024;
 };
@@ -109,7 +112,8 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int cc) {
 // table lookups of four rows are in flight together.
 template <int D>
 __device__ __forceinline__ void rope_tile(uint8_t* tile, int64_t row0, int n_valid,
-                                          const RopeParams& rp, int rt, int* s_pos) {
+                                          const RopeParams& rp, const float2* tab, int rt,
+                                          int* s_pos) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RPP = kRopeThreads / CPR;    // rows per pass
   static_assert(kRopeThreads == kTileM, "one position per thread");
@@ -135,7 +139,7 @@ __device__ __forceinline__ void rope_tile(uint8_t* tile, int64_t row0, int n_val
         const int t = pk & 2047, h = (pk >> 11) & 2047, w = (pk >> 22) & 1023;
         v[u] = *reinterpret_cast<const uint4*>(tile + sw128_chunk(r, cc));
 #pragma unroll
-        for (int e = 0; e < 4; ++e) cs[u][e] = rope_cs(rp, pr[e], t, h, w);
+        for (int e = 0; e < 4; ++e) cs[u][e] = rope_cs_at(tab, pr[e], t, h, w);
       }
     }
 #pragma unroll
@@ -244,7 +248,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar_s = ptx::smem_u32(&b->s_full[qi]);
     const uint32_t bar_p = ptx::smem_u32(&b->p_full[qi]);
     float m = -INFINITY;  // running max of scale*log2(e)*score (lazily updated)
-    float l = 0.f;
+    uint64_t l2 = f2_pack(0.f, 0.f);  // running row sum, two partial sums
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       // warp-uniform decision: tcgen05.ld/st below are warp-collective
@@ -262,15 +266,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int c = 0; c < 128; ++c)
           if (c >= last_valid) s[c] = -INFINITY;
       }
+      // row max: 3-input max in four independent chains
       float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
+      for (int c = 4; c + 8 <= 128; c += 8) {
+        mx0 = max3f(mx0, s[c], s[c + 1]);
+        mx1 = max3f(mx1, s[c + 2], s[c + 3]);
+        mx2 = max3f(mx2, s[c + 4], s[c + 5]);
+        mx3 = max3f(mx3, s[c + 6], s[c + 7]);
       }
-      const float mcand = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+      mx0 = max3f(mx0, s[124], s[125]);
+      mx1 = max3f(mx1, s[126], s[127]);
+      const float mcand = max3f(mx0, mx1, fmaxf(mx2, mx3)) * p.scale_log2;
       const bool raise = mcand > m + kRescaleThreshold;
       if (__any_sync(0xffffffffu, raise && j > 0)) {
         // warp-collective O rescale (lanes that keep their max use factor 1)
@@ -284,26 +291,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * f);
           ptx::tmem_st16(tO + c * 16, ov);
         }
-        l *= f;
+        l2 = f2_mul(l2, f2_pack(f, f));
       }
       if (raise) m = mcand;
-      const float neg_m = -m;
-      float l0 = 0.f, l1 = 0.f;
+      // p = 2^(s * scale * log2(e) - m): packed FFMA2 for the affine part, MUFU ex2,
+      // packed FADD2 for the row sum
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m, -m);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         // P for 32 keys -> 16 packed columns, stored as soon as they are ready
         uint32_t pw[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float e0 = ex2(fmaf(s[32 * q4 + 2 * c], p.scale_log2, neg_m));
-          const float e1 = ex2(fmaf(s[32 * q4 + 2 * c + 1], p.scale_log2, neg_m));
-          l0 += e0;
-          l1 += e1;
+          const uint64_t t2 = f2_fma(f2_pack(s[32 * q4 + 2 * c], s[32 * q4 + 2 * c + 1]), sc2, nm2);
+          float t0, t1;
+          f2_unpack(t2, t0, t1);
+          const float e0 = ex2(t0), e1 = ex2(t1);
+          l2 = f2_add(l2, f2_pack(e0, e1));
           pw[c] = pack_bf16x2(e0, e1);
         }
         ptx::tmem_st16(tS + 16 * q4, pw);
       }
-      l += l0 + l1;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar_p);
@@ -313,6 +321,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ptx::tc_fence_after();
       const int64_t row_in_seq = q_row0 + qi * kTileM + r;
       const bool valid = row_in_seq < seq_len;
+      float l_lo, l_hi;
+      f2_unpack(l2, l_lo, l_hi);
+      const float l = l_lo + l_hi;
       const float inv_l = 1.f / l;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
                       ((seq_start + row_in_seq) * p.H + head) * static_cast<int64_t>(D) * 2;
@@ -468,12 +479,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             : "memory");
         return r != 0;
       };
+      // the cos/sin table is read for every K tile: keep a copy in shared memory when
+      // it fits (L1 is small next to this kernel's shared-memory footprint)
+      const float2* tab = p.rope.table;
+      if (p.rope.n_entries * 8 <= static_cast<int>(L::kTabBytes)) {
+        float2* st = reinterpret_cast<float2*>(smem + L::kTab);
+        for (int i = rt; i < p.rope.n_entries; i += kRopeThreads) st[i] = __ldg(p.rope.table + i);
+        asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");
+        tab = st;
+      }
       if (all_ok(ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort))) {
         for (int qi = 0; qi < 2; ++qi) {
           const int64_t r0 = q_row0 + qi * kTileM;
           const int64_t rem = seq_len - r0;
           const int nv = rem <= 0 ? 0 : (rem >= kTileM ? kTileM : static_cast<int>(rem));
-          rope_tile<D>(smem + (qi ? L::kQ1 : L::kQ0), r0, nv, p.rope, rt, s_pos);
+          rope_tile<D>(smem + (qi ? L::kQ1 : L::kQ0), r0, nv, p.rope, tab, rt, s_pos);
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
@@ -482,7 +502,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!all_ok(ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort))) break;
           const int nv = (j == nk - 1) ? last_valid : kTileN;
           rope_tile<D>(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv, p.rope,
-                       rt, s_pos);
+                       tab, rt, s_pos);
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&b->k_ready[st]));
         }

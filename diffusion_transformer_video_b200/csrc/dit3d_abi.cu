@@ -115,6 +115,7 @@ int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopePara
   rp->d_w = r->d_w;
   rp->off_h = t_ext * (r->d_t / 2);
   rp->off_w = rp->off_h + r->grid_h * (r->d_h / 2);
+  rp->n_entries = rp->off_w + r->grid_w * (r->d_w / 2);
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_tables.find(key);
   if (it != g_tables.end()) {
@@ -122,6 +123,7 @@ int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopePara
     return DIT_OK;
   }
   const int n = rp->off_w + r->grid_w * (r->d_w / 2);
+  rp->n_entries = n;
   std::vector<float2> host(std::max(n, 1));
   const int ext[3] = {t_ext, r->grid_h, r->grid_w};
   const int width[3] = {r->d_t, r->d_h, r->d_w};

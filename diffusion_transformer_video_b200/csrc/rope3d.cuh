@@ -18,6 +18,7 @@ namespace dit3d {
 
 struct RopeParams {
   const float2* table;
+  int32_t n_entries;     // float2 entries in the table
   int32_t grid_h, grid_w;
   int32_t d_t, d_h, d_w;
   int32_t off_h, off_w;  // start (in float2) of the h and w sections; t starts at 0
@@ -55,6 +56,12 @@ __device__ __forceinline__ float2 rope_cs(const RopeParams& rp, const PairRef& p
                                           int w) {
   const int pos = pr.axis == 0 ? t : (pr.axis == 1 ? h : w);
   return __ldg(rp.table + pr.base + pos * pr.stride);
+}
+// Same lookup in a copy of the table (shared memory or global, generic address).
+__device__ __forceinline__ float2 rope_cs_at(const float2* tab, const PairRef& pr, int t, int h,
+                                             int w) {
+  const int pos = pr.axis == 0 ? t : (pr.axis == 1 ? h : w);
+  return tab[pr.base + pos * pr.stride];
 }
 
 // Rotate the 4 pairs of one 16-byte chunk.
