@@ -106,50 +106,24 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int cc) {
   return static_cast<uint32_t>((cc >> 3) * 16384 + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
 }
 
-// Rotate rows [0, n_valid) of one tile in shared memory. Row r of the tile is
-// token (row0 + r) of its sequence. Runs on the kRopeThreads RoPE threads; each
-// thread owns one 16-byte column chunk and walks rows two at a time so the
-// table lookups of four rows are in flight together.
+// Rotate rows [0, n_valid) of one tile in shared memory, in place. Row r of the tile
+// is token (row0 + r) of its sequence; RoPE thread r owns row r: it decodes the
+// row's (t, h, w) once and walks the row's d/8 chunks (a warp then covers 32 rows
+// of one chunk column: no divergence, conflict-free swizzled accesses).
 template <int D>
 __device__ __forceinline__ void rope_tile(uint8_t* tile, int64_t row0, int n_valid,
-                                          const RopeParams& rp, const float2* tab, int rt,
-                                          int* s_pos) {
-  constexpr int CPR = D / 8;                 // 16-byte chunks per row
-  constexpr int RPP = kRopeThreads / CPR;    // rows per pass
-  static_assert(kRopeThreads == kTileM, "one position per thread");
-  {
-    // position of tile row rt, packed t | h << 11 | w << 22 (host checks the ranges)
-    int t = 0, h = 0, w = 0;
-    if (rt < n_valid) token_pos(row0 + rt, rp.grid_h, rp.grid_w, t, h, w);
-    s_pos[rt] = t | (h << 11) | (w << 22);
+                                          const RopeParams& rp, const float2* tab, int rt) {
+  static_assert(kRopeThreads == kTileM, "one tile row per RoPE thread");
+  if (rt >= n_valid) return;
+  // positions inside one sequence fit in 32 bits (rows < 2^31)
+  const int j = static_cast<int>(row0) + rt;
+  const int hw = rp.grid_h * rp.grid_w;
+  const int t = j / hw, rr = j - t * hw, h = rr / rp.grid_w, w = rr - h * rp.grid_w;
+#pragma unroll 4
+  for (int c = 0; c < D / 8; ++c) {
+    uint4* p = reinterpret_cast<uint4*>(tile + sw128_chunk(rt, c));
+    *p = rope_chunk(rp, tab, *p, c, t, h, w);
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");
-  const int cc = rt % CPR;
-  PairRef pr[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) pr[e] = rope_pair_ref(rp, cc * 4 + e);
-  for (int base = rt / CPR; base < n_valid; base += 2 * RPP) {
-    uint4 v[2];
-    float2 cs[2][4];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int r = base + u * RPP;
-      if (r < n_valid) {
-        const int pk = s_pos[r];
-        const int t = pk & 2047, h = (pk >> 11) & 2047, w = (pk >> 22) & 1023;
-        v[u] = *reinterpret_cast<const uint4*>(tile + sw128_chunk(r, cc));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) cs[u][e] = rope_cs_at(tab, pr[e], t, h, w);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int r = base + u * RPP;
-      if (r < n_valid)
-        *reinterpret_cast<uint4*>(tile + sw128_chunk(r, cc)) = rope_rotate_chunk(v[u], cs[u]);
-    }
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");  // s_pos reuse
 }
 
 template <int D>
@@ -163,7 +137,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __shared__ Barriers bars;
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
-  __shared__ int s_pos[kTileM];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -467,42 +440,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // =========================================================== 3D-RoPE warps
     if (p.use_rope) {
       const int rt = tid - kWarpRope0 * 32;
-      // every RoPE thread waits itself (acquiring the TMA data), then all 64 agree
-      // before the named barriers inside rope_tile
-      auto all_ok = [](bool ok) {
-        uint32_t r;
-        asm volatile(
-            "{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\t"
-            "bar.red.and.pred b, 2, %2, a;\n\tselp.u32 %0, 1, 0, b;\n\t}"
-            : "=r"(r)
-            : "r"(static_cast<uint32_t>(ok)), "n"(kRopeThreads)
-            : "memory");
-        return r != 0;
-      };
-      // the cos/sin table is read for every K tile: keep a copy in shared memory when
-      // it fits (L1 is small next to this kernel's shared-memory footprint)
+      // the cos/sin table is read for every K tile: keep a copy in shared memory when it
+      // fits (L1 is small next to this kernel's shared-memory footprint)
       const float2* tab = p.rope.table;
       if (p.rope.n_entries * 8 <= static_cast<int>(L::kTabBytes)) {
-        float2* st = reinterpret_cast<float2*>(smem + L::kTab);
-        for (int i = rt; i < p.rope.n_entries; i += kRopeThreads) st[i] = __ldg(p.rope.table + i);
+        float4* st = reinterpret_cast<float4*>(smem + L::kTab);
+        const float4* src = reinterpret_cast<const float4*>(p.rope.table);
+        for (int i = rt; i < p.rope.n_entries / 2; i += kRopeThreads) st[i] = __ldg(src + i);
         asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");
-        tab = st;
+        tab = reinterpret_cast<const float2*>(st);
       }
-      if (all_ok(ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort))) {
+      if (ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort)) {
         for (int qi = 0; qi < 2; ++qi) {
           const int64_t r0 = q_row0 + qi * kTileM;
           const int64_t rem = seq_len - r0;
           const int nv = rem <= 0 ? 0 : (rem >= kTileM ? kTileM : static_cast<int>(rem));
-          rope_tile<D>(smem + (qi ? L::kQ1 : L::kQ0), r0, nv, p.rope, tab, rt, s_pos);
+          rope_tile<D>(smem + (qi ? L::kQ1 : L::kQ0), r0, nv, p.rope, tab, rt);
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
         for (int j = 0; j < nk; ++j) {
           const int st = j % kKStages, ph = (j / kKStages) & 1;
-          if (!all_ok(ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort))) break;
+          if (!ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort)) break;
           const int nv = (j == nk - 1) ? last_valid : kTileN;
           rope_tile<D>(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv, p.rope,
-                       tab, rt, s_pos);
+                       tab, rt);
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&b->k_ready[st]));
         }

@@ -101,41 +101,60 @@ int validate_rope(const dit_rope3d_desc* r, int32_t d, const std::vector<int64_t
   return DIT_OK;
 }
 
-// Host fp64 -> fp32 (cos, sin) table for the angle (pos + offset) * base^(-2i/d_a).
+// Host fp64 -> fp32 table of (cos, sin) for the angle (pos + offset) * base^(-2i/d_a),
+// chunk-aligned per band as the kernels read it (see rope3d.cuh).
 int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopeParams* rp) {
   int dev = 0;
   cudaGetDevice(&dev);
   uint32_t bb;
   std::memcpy(&bb, &r->base, 4);
   TableKey key{dev, r->grid_h, r->grid_w, r->d_t, r->d_h, r->d_w, t_ext, r->t0, r->h0, r->w0, bb};
+  const int width[3] = {r->d_t, r->d_h, r->d_w};
+  const int ext[3] = {t_ext, r->grid_h, r->grid_w};
+  const int offs[3] = {r->t0, r->h0, r->w0};
+  const int first_pair[3] = {0, r->d_t / 2, (r->d_t + r->d_h) / 2};
+  int off[3], str[3], cf[3], n = 0;
+  for (int a = 0; a < 3; ++a) {
+    const int np = width[a] / 2;
+    off[a] = n;
+    if (np == 0) {
+      str[a] = 0;
+      cf[a] = 0;
+      continue;
+    }
+    cf[a] = first_pair[a] / 4;
+    const int nchunks = (first_pair[a] + np - 1) / 4 - cf[a] + 1;
+    str[a] = 4 * nchunks + 2;  // an odd number of 16-byte units per position
+    n += ext[a] * str[a];
+  }
   rp->grid_h = r->grid_h;
   rp->grid_w = r->grid_w;
-  rp->d_t = r->d_t;
-  rp->d_h = r->d_h;
-  rp->d_w = r->d_w;
-  rp->off_h = t_ext * (r->d_t / 2);
-  rp->off_w = rp->off_h + r->grid_h * (r->d_h / 2);
-  rp->n_entries = rp->off_w + r->grid_w * (r->d_w / 2);
+  rp->p1 = first_pair[1];
+  rp->p2 = first_pair[2];
+  rp->off0 = off[0]; rp->off1 = off[1]; rp->off2 = off[2];
+  rp->str0 = str[0]; rp->str1 = str[1]; rp->str2 = str[2];
+  rp->cf0 = cf[0]; rp->cf1 = cf[1]; rp->cf2 = cf[2];
+  rp->n_entries = n;
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_tables.find(key);
   if (it != g_tables.end()) {
     rp->table = it->second;
     return DIT_OK;
   }
-  const int n = rp->off_w + r->grid_w * (r->d_w / 2);
-  rp->n_entries = n;
-  std::vector<float2> host(std::max(n, 1));
-  const int ext[3] = {t_ext, r->grid_h, r->grid_w};
-  const int width[3] = {r->d_t, r->d_h, r->d_w};
-  const int off[3] = {r->t0, r->h0, r->w0};
-  int at = 0;
-  for (int a = 0; a < 3; ++a)
+  std::vector<float2> host(std::max(n, 2), make_float2(1.f, 0.f));
+  for (int a = 0; a < 3; ++a) {
+    const int np = width[a] / 2;
+    if (np == 0) continue;
     for (int pos = 0; pos < ext[a]; ++pos)
-      for (int i = 0; i < width[a] / 2; ++i) {
+      for (int p = 4 * cf[a]; p < 4 * cf[a] + str[a] - 2; ++p) {
+        const int i = p - first_pair[a];
+        if (i < 0 || i >= np) continue;  // outside the band: identity
         const double theta = std::pow(static_cast<double>(r->base), -2.0 * i / width[a]);
-        const double phi = static_cast<double>(pos + off[a]) * theta;
-        host[at++] = make_float2(static_cast<float>(std::cos(phi)), static_cast<float>(std::sin(phi)));
+        const double phi = static_cast<double>(pos + offs[a]) * theta;
+        host[off[a] + pos * str[a] + (p - 4 * cf[a])] =
+            make_float2(static_cast<float>(std::cos(phi)), static_cast<float>(std::sin(phi)));
       }
+  }
   float2* dptr = nullptr;
   if (cudaMalloc(&dptr, sizeof(float2) * host.size()) != cudaSuccess) return DIT_ERR_ALLOC;
   // pageable source: the copy has consumed `host` when the call returns

@@ -8,9 +8,16 @@
 // pos * base^(-2i/d_a), rotation [[cos, -sin], [sin, cos]], positions counted from
 // 0 at each sequence start plus a constant offset.
 //
-// The cos/sin values come from a table the host fills in fp64 and stores in fp32:
-// three sections, [T_ext][d_t/2], [grid_h][d_h/2], [grid_w][d_w/2], of float2
-// (cos, sin), with the position offsets already folded into the angles.
+// cos/sin come from a table the host fills in fp64 and stores in fp32, laid out so
+// that one 16-byte data chunk (8 bf16 = 4 pairs) needs two 16-byte table reads.
+// For band a (t, h, w) the table holds, per position pos, the (cos, sin) of every
+// pair of the chunks the band touches -- chunk-aligned, pairs outside the band set
+// to the identity (1, 0) -- at float2 index  off_a + pos * stride_a + 4 * (c - cf_a)
+// for chunk c. stride_a is an odd number of 16-byte units, so 32 lanes reading 32
+// different positions hit distinct bank groups. A chunk that straddles a band edge
+// is rotated once per band it touches; the identity entries leave the other
+// band's pairs exact in fp32, so the result equals a single rotation.
+// The position offsets are folded into the angles.
 #pragma once
 #include "common.cuh"
 
@@ -18,30 +25,16 @@ namespace dit3d {
 
 struct RopeParams {
   const float2* table;
-  int32_t n_entries;     // float2 entries in the table
+  int32_t n_entries;          // float2 entries in the table
   int32_t grid_h, grid_w;
-  int32_t d_t, d_h, d_w;
-  int32_t off_h, off_w;  // start (in float2) of the h and w sections; t starts at 0
+  int32_t p1, p2;             // first pair of the h band and of the w band (t starts at 0)
+  int32_t off0, off1, off2;   // first float2 of each band's section
+  int32_t str0, str1, str2;   // float2 entries per position in each section
+  int32_t cf0, cf1, cf2;      // first chunk each band touches
 };
 
-// Table index, for position 0, and per-position stride of pair p (0 <= p < d/2).
-struct PairRef {
-  int32_t axis;    // 0 = t, 1 = h, 2 = w
-  int32_t base;    // index of (pos = 0, this pair)
-  int32_t stride;  // float2 entries per position step
-};
-
-__device__ __forceinline__ PairRef rope_pair_ref(const RopeParams& rp, int p) {
-  const int ht = rp.d_t >> 1, hh = rp.d_h >> 1, hw = rp.d_w >> 1;
-  PairRef r;
-  if (p < ht) {
-    r.axis = 0; r.base = p; r.stride = ht;
-  } else if (p < ht + hh) {
-    r.axis = 1; r.base = rp.off_h + (p - ht); r.stride = hh;
-  } else {
-    r.axis = 2; r.base = rp.off_w + (p - ht - hh); r.stride = hw;
-  }
-  return r;
+__device__ __forceinline__ int rope_band_of_pair(const RopeParams& rp, int p) {
+  return p < rp.p1 ? 0 : (p < rp.p2 ? 1 : 2);
 }
 
 __device__ __forceinline__ void token_pos(int64_t j, int gh, int gw, int& t, int& h, int& w) {
@@ -52,28 +45,40 @@ __device__ __forceinline__ void token_pos(int64_t j, int gh, int gw, int& t, int
   w = r - h * gw;
 }
 
-__device__ __forceinline__ float2 rope_cs(const RopeParams& rp, const PairRef& pr, int t, int h,
-                                          int w) {
-  const int pos = pr.axis == 0 ? t : (pr.axis == 1 ? h : w);
-  return __ldg(rp.table + pr.base + pos * pr.stride);
-}
-// Same lookup in a copy of the table (shared memory or global, generic address).
-__device__ __forceinline__ float2 rope_cs_at(const float2* tab, const PairRef& pr, int t, int h,
-                                             int w) {
-  const int pos = pr.axis == 0 ? t : (pr.axis == 1 ? h : w);
-  return tab[pr.base + pos * pr.stride];
+// Float2 index, in band a's section, of the first pair of chunk c at position pos.
+__device__ __forceinline__ int rope_entry(const RopeParams& rp, int a, int pos, int c) {
+  const int off = a == 0 ? rp.off0 : (a == 1 ? rp.off1 : rp.off2);
+  const int str = a == 0 ? rp.str0 : (a == 1 ? rp.str1 : rp.str2);
+  const int cf = a == 0 ? rp.cf0 : (a == 1 ? rp.cf1 : rp.cf2);
+  return off + pos * str + 4 * (c - cf);
 }
 
-// Rotate the 4 pairs of one 16-byte chunk.
-__device__ __forceinline__ uint4 rope_rotate_chunk(uint4 v, const float2 (&cs)[4]) {
-  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// x0' = x0 cos - x1 sin, x1' = x0 sin + x1 cos on the four fp32 pairs of a chunk.
+__device__ __forceinline__ void rope_rotate4(float (&x)[8], float4 cs01, float4 cs23) {
+  const float c[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+  const float s[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const float x0 = bf16lo(w[e]), x1 = bf16hi(w[e]);
-    const float c = cs[e].x, s = cs[e].y;
-    w[e] = pack_bf16x2(fmaf(x0, c, -x1 * s), fmaf(x0, s, x1 * c));
+    const float x0 = x[2 * e], x1 = x[2 * e + 1];
+    x[2 * e] = fmaf(x0, c[e], -x1 * s[e]);
+    x[2 * e + 1] = fmaf(x0, s[e], x1 * c[e]);
   }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Rotate chunk c (pairs 4c .. 4c+3) of one row at position (t, h, w). `tab` is the
+// table (in global or shared memory, generic address).
+__device__ __forceinline__ uint4 rope_chunk(const RopeParams& rp, const float2* tab, uint4 v, int c,
+                                            int t, int h, int w) {
+  float x[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
+                bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+  const int a_lo = rope_band_of_pair(rp, 4 * c), a_hi = rope_band_of_pair(rp, 4 * c + 3);
+  for (int a = a_lo; a <= a_hi; ++a) {
+    const int pos = a == 0 ? t : (a == 1 ? h : w);
+    const float4* e = reinterpret_cast<const float4*>(tab + rope_entry(rp, a, pos, c));
+    rope_rotate4(x, e[0], e[1]);
+  }
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
 }
 
 // Sequence start of global row `row` (largest s with cu[s] <= row).
@@ -88,9 +93,9 @@ __device__ __forceinline__ int64_t seq_start_of_row(const int32_t* __restrict__ 
   return __ldg(cu + lo);
 }
 
-// Standalone RoPE: one warp per token row. Lane l always handles column chunk
-// l % (D_HEAD/8) of every head, so its four (cos, sin) pairs are fetched once per
-// row and reused for all heads of q and of k.
+// Standalone RoPE: one warp per token row; lane l handles chunk l % (D_HEAD/8) of
+// every head of q and of k, with the same per-chunk procedure as the attention
+// kernel (so both produce the same bits).
 template <int D_HEAD>
 __global__ void __launch_bounds__(256)
 rope3d_qk_kernel(const uint4* q_in, const uint4* k_in, uint4* q_out, uint4* k_out, int64_t rows,
@@ -104,19 +109,13 @@ rope3d_qk_kernel(const uint4* q_in, const uint4* k_in, uint4* q_out, uint4* k_ou
   int t, h, w;
   token_pos(j, rp.grid_h, rp.grid_w, t, h, w);
   const int cc = lane % (D_HEAD / 8);
-  float2 cs[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) cs[e] = rope_cs(rp, rope_pair_ref(rp, cc * 4 + e), t, h, w);
   const int nchunk = H * (D_HEAD / 8);
   const int64_t base = row * nchunk;
-  for (int c = lane; c < nchunk; c += 32) {
-    q_out[base + c] = rope_rotate_chunk(q_in[base + c], cs);
-  }
-  if (k_in != nullptr) {
-    for (int c = lane; c < nchunk; c += 32) {
-      k_out[base + c] = rope_rotate_chunk(k_in[base + c], cs);
-    }
-  }
+  for (int c = lane; c < nchunk; c += 32)
+    q_out[base + c] = rope_chunk(rp, rp.table, q_in[base + c], cc, t, h, w);
+  if (k_in != nullptr)
+    for (int c = lane; c < nchunk; c += 32)
+      k_out[base + c] = rope_chunk(rp, rp.table, k_in[base + c], cc, t, h, w);
 }
 
 }  // namespace dit3d
