@@ -248,6 +248,9 @@ const char* dit_status_string(int status) {
     case DIT_ERR_LAUNCH: return "DIT_ERR_LAUNCH: a CUDA call or kernel launch failed";
     case DIT_ERR_TIMEOUT: return "DIT_ERR_TIMEOUT: a kernel gave up a bounded wait";
     case DIT_ERR_ALLOC: return "DIT_ERR_ALLOC: device allocation for the RoPE table failed";
+    case DIT_ERR_SCRATCH:
+      return "DIT_ERR_SCRATCH: the RoPE table is larger than the fixed array of the "
+             "allocation-free call (65536 entries)";
     default: return "unknown dit_status";
   }
 }
@@ -406,3 +409,134 @@ void dit_shutdown(void) {
 void dit_debug_force_timeout(int enable) { g_force_timeout = enable ? 1 : 0; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free attention
+// dit_attn_fwd_noalloc: the same attention, but the 3D-RoPE cos/sin table lives in a
+// fixed array of device memory that is part of the loaded library, so the call never
+// allocates. The array is shared by every call on a device and holds the last call's
+// table; the host rewrites the whole used range on every call.
+namespace {
+
+constexpr int kNoAllocTableEntries = 65536;  // float2 entries: 512 KiB per device
+static __device__ __align__(256) float2 g_noalloc_rope_table[kNoAllocTableEntries];
+
+std::mutex g_noalloc_mu;
+std::map<int, float2*> g_noalloc_addr;  // per device: the array's device address
+
+// Device address of the array on the current device. The array's name in host code
+// is only a stand-in, so the address is asked from the runtime once per device.
+int noalloc_table_address(float2** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  auto it = g_noalloc_addr.find(dev);
+  if (it == g_noalloc_addr.end()) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_rope_table) != cudaSuccess || ptr == nullptr)
+      return DIT_ERR_LAUNCH;
+    it = g_noalloc_addr.emplace(dev, static_cast<float2*>(ptr)).first;
+  }
+  *out = it->second;
+  return DIT_OK;
+}
+
+// The RoPE table in the layout rope3d.cuh reads, built on the host in fp64 (the same
+// values the cached tables hold), and its section parameters.
+void noalloc_fill_table(const dit_rope3d_desc* r, int t_ext, RopeParams* rp,
+                        std::vector<float2>* host) {
+  const int width[3] = {r->d_t, r->d_h, r->d_w};
+  const int ext[3] = {t_ext, r->grid_h, r->grid_w};
+  const int offs[3] = {r->t0, r->h0, r->w0};
+  const int first_pair[3] = {0, r->d_t / 2, (r->d_t + r->d_h) / 2};
+  int off[3], str[3], cf[3], n = 0;
+  for (int a = 0; a < 3; ++a) {
+    const int np = width[a] / 2;
+    off[a] = n;
+    str[a] = 0;
+    cf[a] = 0;
+    if (np == 0) continue;
+    cf[a] = first_pair[a] / 4;
+    str[a] = 4 * ((first_pair[a] + np - 1) / 4 - cf[a] + 1) + 2;
+    n += ext[a] * str[a];
+  }
+  rp->grid_h = r->grid_h;
+  rp->grid_w = r->grid_w;
+  rp->p1 = first_pair[1];
+  rp->p2 = first_pair[2];
+  rp->off0 = off[0]; rp->off1 = off[1]; rp->off2 = off[2];
+  rp->str0 = str[0]; rp->str1 = str[1]; rp->str2 = str[2];
+  rp->cf0 = cf[0]; rp->cf1 = cf[1]; rp->cf2 = cf[2];
+  rp->n_entries = n;
+  host->assign(std::max(n, 2), make_float2(1.f, 0.f));
+  for (int a = 0; a < 3; ++a) {
+    const int np = width[a] / 2;
+    if (np == 0) continue;
+    for (int pos = 0; pos < ext[a]; ++pos)
+      for (int p = 4 * cf[a]; p < 4 * cf[a] + str[a] - 2; ++p) {
+        const int i = p - first_pair[a];
+        if (i < 0 || i >= np) continue;
+        const double theta = std::pow(static_cast<double>(r->base), -2.0 * i / width[a]);
+        const double phi = static_cast<double>(pos + offs[a]) * theta;
+        (*host)[off[a] + pos * str[a] + (p - 4 * cf[a])] =
+            make_float2(static_cast<float>(std::cos(phi)), static_cast<float>(std::sin(phi)));
+      }
+  }
+}
+
+}  // namespace
+
+extern "C" int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int64_t rows, int32_t H, int32_t d,
+                                    int32_t n_seq, const int32_t* cu_seqlens_dev,
+                                    const int32_t* cu_seqlens_host, float softmax_scale,
+                                    const dit_rope3d_desc* rope, void* stream) {
+  if (!q || !k || !v || !o) return DIT_ERR_NULL;
+  if (rows <= 0 || H <= 0 || H > 65535 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
+  if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return DIT_ERR_ALIGN;
+  std::vector<int64_t> lens;
+  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
+  int t_ext = 0;
+  if (rope)
+    if (int s = validate_rope(rope, d, lens, &t_ext)) return s;
+  if (int s = check_device()) return s;
+  auto st = static_cast<cudaStream_t>(stream);
+
+  attn::Params prm{};
+  prm.cu_seqlens = cu_seqlens_dev;
+  prm.n_seq = n_seq;
+  prm.H = H;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.force_timeout = g_force_timeout;
+  int64_t n_work = 0;
+  if (cu_seqlens_dev == nullptr) {
+    prm.dense_len = rows / n_seq;
+    prm.pairs_per_dense_seq =
+        static_cast<int32_t>((prm.dense_len + 2 * attn::kTileM - 1) / (2 * attn::kTileM));
+    n_work = static_cast<int64_t>(prm.pairs_per_dense_seq) * n_seq;
+  } else {
+    for (int64_t L : lens) n_work += (L + 2 * attn::kTileM - 1) / (2 * attn::kTileM);
+  }
+  if (n_work == 0) return DIT_OK;
+  if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
+  if (rope) {
+    std::vector<float2> host;
+    noalloc_fill_table(rope, t_ext, &prm.rope, &host);
+    if (prm.rope.n_entries > kNoAllocTableEntries) return DIT_ERR_SCRATCH;
+    float2* table = nullptr;
+    if (int s = noalloc_table_address(&table)) return s;
+    // pageable source: the copy has consumed `host` when the call returns
+    if (cudaMemcpyAsync(table, host.data(), sizeof(float2) * host.size(), cudaMemcpyHostToDevice,
+                        st) != cudaSuccess)
+      return DIT_ERR_LAUNCH;
+    prm.use_rope = 1;
+    prm.rope.table = table;
+  }
+  if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+  return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+}

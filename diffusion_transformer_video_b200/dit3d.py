@@ -18,11 +18,12 @@ LIB_PATH = os.path.join(_PKG, "libdit3d.so")
 DIT_OK = 0
 STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_ALIGN",
                 4: "DIT_ERR_SEQLENS", 5: "DIT_ERR_DEVICE", 6: "DIT_ERR_LAUNCH",
-                7: "DIT_ERR_TIMEOUT", 8: "DIT_ERR_ALLOC"}
+                7: "DIT_ERR_TIMEOUT", 8: "DIT_ERR_ALLOC", 9: "DIT_ERR_SCRATCH"}
 
 # every symbol include/dit3d.h declares
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
-           "dit_check_device", "dit_status_string", "dit_shutdown", "dit_debug_force_timeout")
+           "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
+           "dit_debug_force_timeout")
 
 
 class DitError(RuntimeError):
@@ -62,6 +63,9 @@ def lib():
                                     ctypes.POINTER(RopeDesc), P]
         L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
                                    ctypes.POINTER(RopeDesc), P]
+        L.dit_attn_fwd_noalloc.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
+                                           ctypes.POINTER(RopeDesc), P]
+        L.dit_attn_fwd_noalloc.restype = ctypes.c_int
         L.dit_check_device.argtypes = [P]
         L.dit_status_string.argtypes = [ctypes.c_int]
         L.dit_status_string.restype = ctypes.c_char_p

@@ -51,7 +51,8 @@ enum dit_status {
   DIT_ERR_DEVICE = 5,   /* current device is not sm_100 (B200 class)                     */
   DIT_ERR_LAUNCH = 6,   /* a CUDA call or kernel launch failed                          */
   DIT_ERR_TIMEOUT = 7,  /* a kernel's bounded wait expired (reported by dit_check_device) */
-  DIT_ERR_ALLOC = 8     /* the RoPE table cache could not allocate device memory        */
+  DIT_ERR_ALLOC = 8,    /* the RoPE table cache could not allocate device memory        */
+  DIT_ERR_SCRATCH = 9   /* dit_attn_fwd_noalloc: the RoPE table exceeds its fixed array  */
 };
 
 /* 3D-RoPE descriptor (DiT page, section "3D-RoPE e atencao espaco-temporal"):
@@ -120,6 +121,31 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
                  const int32_t* cu_seqlens_host, float softmax_scale, const dit_rope3d_desc* rope,
                  void* stream);
+
+/* Allocation-free variant of dit_attn_fwd (no counterpart in the source pages).
+ * Same arguments, layouts, results and errors as dit_attn_fwd; the difference is
+ * where the 3D-RoPE cos/sin table lives. dit_attn_fwd allocates it with cudaMalloc
+ * on first use and caches it; this call instead writes it (host-computed, the same
+ * values) into a fixed array of device memory that belongs to the loaded library,
+ * so it never calls cudaMalloc, cudaFree or any allocating routine. It is meant for
+ * callers that must not allocate device memory while they run: processes that hand
+ * all device memory to their own pool or allocator up front, memory-capped serving
+ * workers, and latency-critical paths that cannot afford cudaMalloc's implicit
+ * device synchronisation.
+ *   - The array holds at most 65536 (cos, sin) pairs (512 KiB); a larger table (long
+ *     videos or large patch grids) returns DIT_ERR_SCRATCH and launches nothing.
+ *   - Every GPU that loads the library holds the array until the process exits.
+ *   - The first call on a device looks up the array's device address (a runtime
+ *     query, no allocation); make that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's table:
+ *     each call rewrites the whole range it uses (a copy on `stream` before the
+ *     kernel), so calls whose work overlaps on the GPU (different streams without
+ *     ordering) race on the array and must be serialised by the caller.
+ *   - With rope == NULL no table is involved and the call is dit_attn_fwd exactly. */
+int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                         const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                         float softmax_scale, const dit_rope3d_desc* rope, void* stream);
 
 /* Waits for `stream`, then reads and clears the library's device error word.
  * Returns DIT_ERR_TIMEOUT if any kernel gave up a bounded wait since the last
