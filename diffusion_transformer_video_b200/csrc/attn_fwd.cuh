@@ -106,23 +106,97 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int cc) {
   return static_cast<uint32_t>((cc >> 3) * 16384 + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
 }
 
+// 16-byte shared-memory load / store. The loads carry no memory clobber, so the
+// compiler may hoist the next chunks' loads above this chunk's store (the table and
+// the chunks a thread touches never overlap).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float4 lds128f(uint32_t a) {
+  float4 v;
+  asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 rope_apply(uint4 v, float4 e0, float4 e1) {
+  float x[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
+                bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+  rope_rotate4(x, e0, e1);
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
+}
+
 // Rotate rows [0, n_valid) of one tile in shared memory, in place. Row r of the tile
 // is token (row0 + r) of its sequence; RoPE thread r owns row r: it decodes the
 // row's (t, h, w) once and walks the row's d/8 chunks (a warp then covers 32 rows
 // of one chunk column: no divergence, conflict-free swizzled accesses).
+// Pass 1 rotates every chunk by the band of its first pair, four chunks at a time
+// with all their loads issued first; pass 2 applies the other band(s) to the few
+// chunks that straddle a band edge. Every pair is turned exactly once (identity
+// entries elsewhere, and the bf16 round trip of an untouched value is exact), so the
+// result equals the standalone kernel's single rotation bit for bit.
 template <int D>
-__device__ __forceinline__ void rope_tile(uint8_t* tile, int64_t row0, int n_valid,
-                                          const RopeParams& rp, const float2* tab, int rt) {
+__device__ __forceinline__ void rope_tile_smem(uint32_t tile, int64_t row0, int n_valid,
+                                               const RopeParams& rp, uint32_t tab, int rt) {
   static_assert(kRopeThreads == kTileM, "one tile row per RoPE thread");
   if (rt >= n_valid) return;
-  // positions inside one sequence fit in 32 bits (rows < 2^31)
+  const int j = static_cast<int>(row0) + rt;  // positions inside a sequence fit in 32 bits
+  const int hw = rp.grid_h * rp.grid_w;
+  const int t = j / hw, rr = j - t * hw, h = rr / rp.grid_w, w = rr - h * rp.grid_w;
+  const uint32_t row_t = tab + 8u * static_cast<uint32_t>(rp.off0 + t * rp.str0 - 4 * rp.cf0);
+  const uint32_t row_h = tab + 8u * static_cast<uint32_t>(rp.off1 + h * rp.str1 - 4 * rp.cf1);
+  const uint32_t row_w = tab + 8u * static_cast<uint32_t>(rp.off2 + w * rp.str2 - 4 * rp.cf2);
+#pragma unroll
+  for (int c0 = 0; c0 < D / 8; c0 += 4) {
+    uint4 v[4];
+    float4 e0[4], e1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u;
+      const int a = rope_band_of_pair(rp, 4 * c);
+      const uint32_t e = (a == 0 ? row_t : (a == 1 ? row_h : row_w)) + 32u * c;
+      v[u] = lds128(tile + sw128_chunk(rt, c));
+      e0[u] = lds128f(e);
+      e1[u] = lds128f(e + 16u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sts128(tile + sw128_chunk(rt, c0 + u), rope_apply(v[u], e0[u], e1[u]));
+  }
+  // pass 2: chunks across a band edge get the rotation of their later band(s)
+  const int cs1 = (rp.p1 & 3) ? (rp.p1 >> 2) : -1;   // chunk holding the t/h edge
+  const int cs2 = (rp.p2 & 3) ? (rp.p2 >> 2) : -1;   // chunk holding the h/w edge
+#pragma unroll 1
+  for (int k = 0; k < 2; ++k) {
+    const int c = k ? cs2 : cs1;
+    if (c < 0 || (k && c == cs1)) continue;
+    const int a_lo = rope_band_of_pair(rp, 4 * c), a_hi = rope_band_of_pair(rp, 4 * c + 3);
+    for (int a = a_lo + 1; a <= a_hi; ++a) {
+      const uint32_t e = (a == 1 ? row_h : row_w) + 32u * c;
+      const uint32_t ad = tile + sw128_chunk(rt, c);
+      sts128(ad, rope_apply(lds128(ad), lds128f(e), lds128f(e + 16u)));
+    }
+  }
+}
+
+// Same rotation with the table in global memory (tables larger than the shared copy).
+template <int D>
+__device__ __forceinline__ void rope_tile_global(uint8_t* tile, int64_t row0, int n_valid,
+                                                 const RopeParams& rp, int rt) {
+  if (rt >= n_valid) return;
   const int j = static_cast<int>(row0) + rt;
   const int hw = rp.grid_h * rp.grid_w;
   const int t = j / hw, rr = j - t * hw, h = rr / rp.grid_w, w = rr - h * rp.grid_w;
-#pragma unroll 4
+#pragma unroll 1
   for (int c = 0; c < D / 8; ++c) {
     uint4* p = reinterpret_cast<uint4*>(tile + sw128_chunk(rt, c));
-    *p = rope_chunk(rp, tab, *p, c, t, h, w);
+    *p = rope_chunk(rp, rp.table, *p, c, t, h, w);
   }
 }
 
@@ -442,20 +516,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int rt = tid - kWarpRope0 * 32;
       // the cos/sin table is read for every K tile: keep a copy in shared memory when it
       // fits (L1 is small next to this kernel's shared-memory footprint)
-      const float2* tab = p.rope.table;
-      if (p.rope.n_entries * 8 <= static_cast<int>(L::kTabBytes)) {
+      const bool tab_in_smem = p.rope.n_entries * 8 <= static_cast<int>(L::kTabBytes);
+      if (tab_in_smem) {
         float4* st = reinterpret_cast<float4*>(smem + L::kTab);
         const float4* src = reinterpret_cast<const float4*>(p.rope.table);
         for (int i = rt; i < p.rope.n_entries / 2; i += kRopeThreads) st[i] = __ldg(src + i);
         asm volatile("bar.sync 1, %0;" ::"n"(kRopeThreads) : "memory");
-        tab = reinterpret_cast<const float2*>(st);
       }
+      const uint32_t tab = ptx::smem_u32(smem + L::kTab);
+      auto rope_tile = [&](uint8_t* tile, int64_t row0, int nv) {
+        if (tab_in_smem) rope_tile_smem<D>(ptx::smem_u32(tile), row0, nv, p.rope, tab, rt);
+        else rope_tile_global<D>(tile, row0, nv, p.rope, rt);
+      };
       if (ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort)) {
         for (int qi = 0; qi < 2; ++qi) {
           const int64_t r0 = q_row0 + qi * kTileM;
           const int64_t rem = seq_len - r0;
           const int nv = rem <= 0 ? 0 : (rem >= kTileM ? kTileM : static_cast<int>(rem));
-          rope_tile<D>(smem + (qi ? L::kQ1 : L::kQ0), r0, nv, p.rope, tab, rt);
+          rope_tile(smem + (qi ? L::kQ1 : L::kQ0), r0, nv);
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
@@ -463,8 +541,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int st = j % kKStages, ph = (j / kKStages) & 1;
           if (!ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort)) break;
           const int nv = (j == nk - 1) ? last_valid : kTileN;
-          rope_tile<D>(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv, p.rope,
-                       tab, rt);
+          rope_tile(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv);
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&b->k_ready[st]));
         }
