@@ -34,9 +34,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
 UNIT = "TFLOP/s"
-# dram__bytes_read.sum + dram__bytes_write.sum of one attention launch from an ncu capture,
-# per query/key token pair and head (scaled to the workload); None until captured.
-ATTN_DRAM_BYTES_PER_LAUNCH = None
+# DRAM bytes of one fused-RoPE attention launch per head, from an ncu capture of the 480P
+# geometry with 16 heads (528 MB / 16; profiles/attn_fwd_fused_rope_480p.md). Heads are
+# independent, so the traffic of the 480P launch is this times its head count. Other
+# workloads have no capture: their traffic is reported as null.
+ATTN_DRAM_BYTES_PER_HEAD_480P = 528.09e6 / 16
 
 
 def _peaks():
@@ -101,23 +103,28 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_oracle_attention(w, inp, n_rows: int, seed: int = 0):
+def widen_qkv(inp):
+    """The oracle's fp64 copies of q, k, v (made once, outside any timed region)."""
+    from diffusion_transformer_video_b200 import workloads as wl
+    return tuple(wl.bf16_bits_to_f64(inp[n]) for n in ("q", "k", "v"))
+
+
+def cpu_oracle_attention(w, qkv64, n_rows: int, seed: int = 0):
     """Time the oracle's 3D-RoPE attention on `n_rows` sampled query rows (all heads, all
     keys of their sequences). Returns (TFLOP/s, seconds, sample description, threads)."""
     import oracle
-    from diffusion_transformer_video_b200 import workloads as wl
     rng = np.random.default_rng([seed, 77])
     rows = np.sort(rng.choice(w.rows, size=n_rows, replace=False)).astype(np.int64)
     cu = w.cu_seqlens
-    q, k, v = (wl.bf16_bits_to_f64(inp[n]) for n in ("q", "k", "v"))
+    q, k, v = qkv64
     t0 = time.perf_counter()
     oracle.attn_fwd(q, k, v, cu, qrows=rows, rope=w.rope_desc())
     dt = time.perf_counter() - t0
     seq_of = np.searchsorted(cu, rows, side="right") - 1
     flops = float(sum(4.0 * (cu[s + 1] - cu[s]) * w.head_dim * w.heads for s in seq_of))
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = (f"{n_rows} query rows x {w.heads} heads of {w.name}, all keys of their sequence, "
-              f"3D-RoPE of full q and k included (fp64, OpenMP)")
+    sample = (f"{n_rows} query rows x {w.heads} heads of {w.name}, all keys of their sequence; "
+              f"the oracle's 3D-RoPE of the full q and k is inside the timed call (fp64, OpenMP)")
     return flops / dt / 1e12, dt, sample, threads
 
 
@@ -127,10 +134,11 @@ def run_reference(args, rank, world):
         return
     w = wl.get_workload(args.workload, args.seed)
     inp = wl.make_inputs(w, args.seed, which=("q", "k", "v"))
+    qkv64 = widen_qkv(inp)
     n_rows = args.ref_rows
     vals = []
     for i in range(args.warmup + args.steps):
-        tf, dt, sample, threads = cpu_oracle_attention(w, inp, n_rows, seed=args.seed + i)
+        tf, dt, sample, threads = cpu_oracle_attention(w, qkv64, n_rows, seed=args.seed + i)
         if i >= args.warmup:
             vals.append((tf, dt))
     value = statistics.mean(v for v, _ in vals)
@@ -321,7 +329,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, dt, sample, threads = cpu_oracle_attention(w, inp, args.cpu_rows, args.seed)
+        tf, dt, sample, threads = cpu_oracle_attention(w, widen_qkv(inp), args.cpu_rows, args.seed)
         cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
                "seconds": dt}
 
@@ -342,7 +350,8 @@ def main():
             "roofline": {"bound": "tensor", "achieved": att_tflops,
                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": att_tflops / pk["bf16_tflops_sustained"],
-                         "traffic": ATTN_DRAM_BYTES_PER_LAUNCH,
+                         "traffic": (ATTN_DRAM_BYTES_PER_HEAD_480P * H
+                                     if w.name == "480p" and args.rope_mode == "fused" else None),
                          "kernel": {"fused": "dit_attn_fwd (fused 3D-RoPE)",
                                     "prepass": "dit_rope3d_qk + dit_attn_fwd",
                                     "none": "dit_attn_fwd without RoPE"}[args.rope_mode],
