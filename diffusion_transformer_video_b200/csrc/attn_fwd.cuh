@@ -90,7 +90,7 @@ struct Barriers {
   uint64_t q_full, q_ready;
   uint64_t k_full[kKStages], k_ready[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], p_half[2], p_full[2];  // P of keys 0-63 / all 128 keys in TMEM
   uint64_t o_final, drain;
 };
 
@@ -262,6 +262,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(ptx::smem_u32(&b->s_full[i]), 1);
+      ptx::mbar_init(ptx::smem_u32(&b->p_half[i]), kTileM);
       ptx::mbar_init(ptx::smem_u32(&b->p_full[i]), kTileM);
     }
     ptx::mbar_init(ptx::smem_u32(&b->o_final), 1);
@@ -294,6 +295,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tO = tmem + lane_base + col_o(qi);
     const uint32_t bar_s = ptx::smem_u32(&b->s_full[qi]);
     const uint32_t bar_p = ptx::smem_u32(&b->p_full[qi]);
+    const uint32_t bar_ph = ptx::smem_u32(&b->p_half[qi]);
     float m = -INFINITY;  // running max of scale*log2(e)*score (lazily updated)
     uint64_t l2 = f2_pack(0.f, 0.f);  // running row sum, two partial sums
     bool ok = true;
@@ -358,6 +360,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           pw[c] = pack_bf16x2(e0, e1);
         }
         ptx::tmem_st16(tS + 16 * q4, pw);
+        if (q4 == 1) {
+          // keys 0-63 are in TMEM: the MMA warp may start O += P V on them
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bar_ph);
+        }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -459,13 +467,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         ptx::umma_commit(ptx::smem_u32(&b->s_full[qi]));
       };
-      auto pv = [&](int qi, int st, bool acc) {
+      // O_qi (+)= P_qi V over keys [64 * half, 64 * half + 64)
+      auto pv = [&](int qi, int st, bool acc, int half) {
         const uint32_t va = sbase + L::kV + st * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk)
+        for (int k4 = 0; k4 < kTileN / 32; ++k4) {
+          const int kk = half * (kTileN / 32) + k4;
           ptx::umma_ts(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
                        ptx::make_smem_desc(va + kk * 2048, 16384, 1024, ptx::kSwizzle128B),
                        idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      // both halves, the second once the softmax has stored all of P
+      auto pv_tile = [&](int qi, int st, bool acc, int j) -> bool {
+        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_half[qi]), j & 1, abort)) return false;
+        ptx::tc_fence_after();
+        pv(qi, st, acc, 0);
+        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_full[qi]), j & 1, abort)) return false;
+        ptx::tc_fence_after();
+        pv(qi, st, acc, 1);
+        return true;
       };
       const uint32_t q_wait = ptx::smem_u32(p.use_rope ? &b->q_ready : &b->q_full);
       bool ok = ptx::mbar_wait(q_wait, 0, abort);
@@ -482,9 +503,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int ks1 = (j + 1) % kKStages, kph1 = ((j + 1) / kKStages) & 1;
         const bool more = j + 1 < nk;
         if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[vs]), vph, abort))) break;
-        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->p_full[0]), j & 1, abort))) break;
-        ptx::tc_fence_after();
-        pv(0, vs, j > 0);
+        if (!(ok = pv_tile(0, vs, j > 0, j))) break;
         if (more) {
           if (!(ok = ptx::mbar_wait(
                     ptx::smem_u32(p.use_rope ? &b->k_ready[ks1] : &b->k_full[ks1]), kph1, abort)))
@@ -492,9 +511,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           ptx::tc_fence_after();
           qk(0, ks1);
         }
-        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->p_full[1]), j & 1, abort))) break;
-        ptx::tc_fence_after();
-        pv(1, vs, j > 0);
+        if (!(ok = pv_tile(1, vs, j > 0, j))) break;
         ptx::umma_commit(ptx::smem_u32(&b->v_empty[vs]));
         if (more) {
           qk(1, ks1);

@@ -101,27 +101,18 @@ int validate_rope(const dit_rope3d_desc* r, int32_t d, const std::vector<int64_t
   return DIT_OK;
 }
 
-// Host fp64 -> fp32 table of (cos, sin) for the angle (pos + offset) * base^(-2i/d_a),
-// chunk-aligned per band as the kernels read it (see rope3d.cuh).
-int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopeParams* rp) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  uint32_t bb;
-  std::memcpy(&bb, &r->base, 4);
-  TableKey key{dev, r->grid_h, r->grid_w, r->d_t, r->d_h, r->d_w, t_ext, r->t0, r->h0, r->w0, bb};
+// Section parameters of the RoPE table (layout described in rope3d.cuh).
+void rope_table_layout(const dit_rope3d_desc* r, int t_ext, RopeParams* rp) {
   const int width[3] = {r->d_t, r->d_h, r->d_w};
   const int ext[3] = {t_ext, r->grid_h, r->grid_w};
-  const int offs[3] = {r->t0, r->h0, r->w0};
   const int first_pair[3] = {0, r->d_t / 2, (r->d_t + r->d_h) / 2};
   int off[3], str[3], cf[3], n = 0;
   for (int a = 0; a < 3; ++a) {
     const int np = width[a] / 2;
     off[a] = n;
-    if (np == 0) {
-      str[a] = 0;
-      cf[a] = 0;
-      continue;
-    }
+    str[a] = 0;
+    cf[a] = 0;
+    if (np == 0) continue;
     cf[a] = first_pair[a] / 4;
     const int nchunks = (first_pair[a] + np - 1) / 4 - cf[a] + 1;
     str[a] = 4 * nchunks + 2;  // an odd number of 16-byte units per position
@@ -135,13 +126,22 @@ int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopePara
   rp->str0 = str[0]; rp->str1 = str[1]; rp->str2 = str[2];
   rp->cf0 = cf[0]; rp->cf1 = cf[1]; rp->cf2 = cf[2];
   rp->n_entries = n;
-  std::lock_guard<std::mutex> lk(g_mu);
-  auto it = g_tables.find(key);
-  if (it != g_tables.end()) {
-    rp->table = it->second;
-    return DIT_OK;
-  }
-  std::vector<float2> host(std::max(n, 2), make_float2(1.f, 0.f));
+}
+
+// Host values of the table: cos/sin of the angle (pos + offset) * base^(-2i/d_a) in
+// fp64, stored fp32; a chunk's floats are (cos p0, cos p1, sin p0, sin p1, cos p2,
+// cos p3, sin p2, sin p3), pairs outside the band hold the identity.
+void rope_table_values(const dit_rope3d_desc* r, int t_ext, const RopeParams& rp,
+                       std::vector<float2>* out) {
+  const int width[3] = {r->d_t, r->d_h, r->d_w};
+  const int ext[3] = {t_ext, r->grid_h, r->grid_w};
+  const int offs[3] = {r->t0, r->h0, r->w0};
+  const int first_pair[3] = {0, r->d_t / 2, (r->d_t + r->d_h) / 2};
+  const int off[3] = {rp.off0, rp.off1, rp.off2}, str[3] = {rp.str0, rp.str1, rp.str2},
+            cf[3] = {rp.cf0, rp.cf1, rp.cf2};
+  out->assign(std::max(rp.n_entries, 2), make_float2(1.f, 0.f));  // (1,1,0,0) per couple
+  float* f = reinterpret_cast<float*>(out->data());
+  for (size_t i = 0; i < 2 * out->size(); ++i) f[i] = (i & 2) ? 0.f : 1.f;
   for (int a = 0; a < 3; ++a) {
     const int np = width[a] / 2;
     if (np == 0) continue;
@@ -151,10 +151,31 @@ int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopePara
         if (i < 0 || i >= np) continue;  // outside the band: identity
         const double theta = std::pow(static_cast<double>(r->base), -2.0 * i / width[a]);
         const double phi = static_cast<double>(pos + offs[a]) * theta;
-        host[off[a] + pos * str[a] + (p - 4 * cf[a])] =
-            make_float2(static_cast<float>(std::cos(phi)), static_cast<float>(std::sin(phi)));
+        const int e = p - 4 * cf[a];                        // pair index from the row start
+        float* chunk = f + 2 * (off[a] + pos * str[a]) + 8 * (e >> 2);
+        const int u = (e & 3) >> 1, w = e & 1;              // couple, pair within couple
+        chunk[4 * u + w] = static_cast<float>(std::cos(phi));
+        chunk[4 * u + 2 + w] = static_cast<float>(std::sin(phi));
       }
   }
+}
+
+// Cached device copy of the table for a descriptor (allocated once per device).
+int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopeParams* rp) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  uint32_t bb;
+  std::memcpy(&bb, &r->base, 4);
+  TableKey key{dev, r->grid_h, r->grid_w, r->d_t, r->d_h, r->d_w, t_ext, r->t0, r->h0, r->w0, bb};
+  rope_table_layout(r, t_ext, rp);
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_tables.find(key);
+  if (it != g_tables.end()) {
+    rp->table = it->second;
+    return DIT_OK;
+  }
+  std::vector<float2> host;
+  rope_table_values(r, t_ext, *rp, &host);
   float2* dptr = nullptr;
   if (cudaMalloc(&dptr, sizeof(float2) * host.size()) != cudaSuccess) return DIT_ERR_ALLOC;
   // pageable source: the copy has consumed `host` when the call returns
@@ -440,49 +461,6 @@ int noalloc_table_address(float2** out) {
   return DIT_OK;
 }
 
-// The RoPE table in the layout rope3d.cuh reads, built on the host in fp64 (the same
-// values the cached tables hold), and its section parameters.
-void noalloc_fill_table(const dit_rope3d_desc* r, int t_ext, RopeParams* rp,
-                        std::vector<float2>* host) {
-  const int width[3] = {r->d_t, r->d_h, r->d_w};
-  const int ext[3] = {t_ext, r->grid_h, r->grid_w};
-  const int offs[3] = {r->t0, r->h0, r->w0};
-  const int first_pair[3] = {0, r->d_t / 2, (r->d_t + r->d_h) / 2};
-  int off[3], str[3], cf[3], n = 0;
-  for (int a = 0; a < 3; ++a) {
-    const int np = width[a] / 2;
-    off[a] = n;
-    str[a] = 0;
-    cf[a] = 0;
-    if (np == 0) continue;
-    cf[a] = first_pair[a] / 4;
-    str[a] = 4 * ((first_pair[a] + np - 1) / 4 - cf[a] + 1) + 2;
-    n += ext[a] * str[a];
-  }
-  rp->grid_h = r->grid_h;
-  rp->grid_w = r->grid_w;
-  rp->p1 = first_pair[1];
-  rp->p2 = first_pair[2];
-  rp->off0 = off[0]; rp->off1 = off[1]; rp->off2 = off[2];
-  rp->str0 = str[0]; rp->str1 = str[1]; rp->str2 = str[2];
-  rp->cf0 = cf[0]; rp->cf1 = cf[1]; rp->cf2 = cf[2];
-  rp->n_entries = n;
-  host->assign(std::max(n, 2), make_float2(1.f, 0.f));
-  for (int a = 0; a < 3; ++a) {
-    const int np = width[a] / 2;
-    if (np == 0) continue;
-    for (int pos = 0; pos < ext[a]; ++pos)
-      for (int p = 4 * cf[a]; p < 4 * cf[a] + str[a] - 2; ++p) {
-        const int i = p - first_pair[a];
-        if (i < 0 || i >= np) continue;
-        const double theta = std::pow(static_cast<double>(r->base), -2.0 * i / width[a]);
-        const double phi = static_cast<double>(pos + offs[a]) * theta;
-        (*host)[off[a] + pos * str[a] + (p - 4 * cf[a])] =
-            make_float2(static_cast<float>(std::cos(phi)), static_cast<float>(std::sin(phi)));
-      }
-  }
-}
-
 }  // namespace
 
 extern "C" int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
@@ -526,7 +504,8 @@ extern "C" int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
   if (rope) {
     std::vector<float2> host;
-    noalloc_fill_table(rope, t_ext, &prm.rope, &host);
+    rope_table_layout(rope, t_ext, &prm.rope);
+    rope_table_values(rope, t_ext, prm.rope, &host);
     if (prm.rope.n_entries > kNoAllocTableEntries) return DIT_ERR_SCRATCH;
     float2* table = nullptr;
     if (int s = noalloc_table_address(&table)) return s;

@@ -10,13 +10,15 @@
 //
 // cos/sin come from a table the host fills in fp64 and stores in fp32, laid out so
 // that one 16-byte data chunk (8 bf16 = 4 pairs) needs two 16-byte table reads.
-// For band a (t, h, w) the table holds, per position pos, the (cos, sin) of every
-// pair of the chunks the band touches -- chunk-aligned, pairs outside the band set
-// to the identity (1, 0) -- at float2 index  off_a + pos * stride_a + 4 * (c - cf_a)
-// for chunk c. stride_a is an odd number of 16-byte units, so 32 lanes reading 32
-// different positions hit distinct bank groups. A chunk that straddles a band edge
-// is rotated once per band it touches; the identity entries leave the other
-// band's pairs exact in fp32, so the result equals a single rotation.
+// For band a (t, h, w) the table holds, per position pos, the values of every pair
+// of the chunks the band touches -- chunk-aligned, pairs outside the band set to the
+// identity (cos 1, sin 0) -- starting at float2 index  off_a + pos * stride_a +
+// 4 * (c - cf_a) for chunk c, as (cos p0, cos p1, sin p0, sin p1, cos p2, cos p3,
+// sin p2, sin p3): each pair couple's cosines and sines are adjacent, ready for
+// packed f32x2 arithmetic. stride_a is an odd number of 16-byte units, so 32 lanes
+// reading 32 different positions hit distinct bank groups. A chunk that straddles a
+// band edge is rotated once per band it touches; the identity entries leave the
+// other band's pairs exact in fp32, so the result equals a single rotation.
 // The position offsets are folded into the angles.
 #pragma once
 #include "common.cuh"
@@ -53,16 +55,23 @@ __device__ __forceinline__ int rope_entry(const RopeParams& rp, int a, int pos, 
   return off + pos * str + 4 * (c - cf);
 }
 
-// x0' = x0 cos - x1 sin, x1' = x0 sin + x1 cos on the four fp32 pairs of a chunk.
-__device__ __forceinline__ void rope_rotate4(float (&x)[8], float4 cs01, float4 cs23) {
-  const float c[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-  const float s[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float x0 = x[2 * e], x1 = x[2 * e + 1];
-    x[2 * e] = fmaf(x0, c[e], -x1 * s[e]);
-    x[2 * e + 1] = fmaf(x0, s[e], x1 * c[e]);
-  }
+// x0' = x0 cos - x1 sin, x1' = x0 sin + x1 cos for the two pairs (a0, a1), (b0, b1) of
+// a couple, with f = (cos_a, cos_b, sin_a, sin_b), in packed f32x2 arithmetic (the
+// same roundings as the scalar fmaf(x0, c, -(x1 s)) and fmaf(x0, s, x1 c)).
+__device__ __forceinline__ void rope_rotate_couple(float& a0, float& a1, float& b0, float& b1,
+                                                   float4 f) {
+  const uint64_t X0 = f2_pack(a0, b0), X1 = f2_pack(a1, b1);
+  const uint64_t C = f2_pack(f.x, f.y), S = f2_pack(f.z, f.w);
+  const uint64_t o0 = f2_fma(X0, C, f2_mul(X1, f2_neg(S)));
+  const uint64_t o1 = f2_fma(X0, S, f2_mul(X1, C));
+  f2_unpack(o0, a0, b0);
+  f2_unpack(o1, a1, b1);
+}
+
+// Rotate the four fp32 pairs of a chunk, (x[0], x[1]) .. (x[6], x[7]).
+__device__ __forceinline__ void rope_rotate4(float (&x)[8], float4 f01, float4 f23) {
+  rope_rotate_couple(x[0], x[1], x[2], x[3], f01);
+  rope_rotate_couple(x[4], x[5], x[6], x[7], f23);
 }
 
 // Rotate chunk c (pairs 4c .. 4c+3) of one row at position (t, h, w). `tab` is the
