@@ -192,6 +192,8 @@ def main():
                     help="fused: RoPE inside the attention kernel (the product path); prepass: "
                          "dit_rope3d_qk into scratch then attention; none: attention alone "
                          "(not the workload, a kernel-speed reference)")
+    ap.add_argument("--attn-variant", type=int, default=0, choices=[0, 1],
+                    help="0: single-CTA attention kernel; 1: CTA-pair (cta_group::2) kernel")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (smaller cases for profiling)")
     args = ap.parse_args()
@@ -219,6 +221,7 @@ def main():
         if world > 1:
             dist.barrier()
 
+    dit3d.dit_set_attn_variant(args.attn_variant)
     w = wl.get_workload(args.workload, args.seed)
     if args.heads:
         import dataclasses
@@ -352,6 +355,7 @@ def main():
                          "frac": att_tflops / pk["bf16_tflops_sustained"],
                          "traffic": (ATTN_DRAM_BYTES_PER_HEAD_480P * H
                                      if w.name == "480p" and args.rope_mode == "fused" else None),
+                         "attn_variant": ["single CTA", "CTA pair (cta_group::2)"][args.attn_variant],
                          "kernel": {"fused": "dit_attn_fwd (fused 3D-RoPE)",
                                     "prepass": "dit_rope3d_qk + dit_attn_fwd",
                                     "none": "dit_attn_fwd without RoPE"}[args.rope_mode],

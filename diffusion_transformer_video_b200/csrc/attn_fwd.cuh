@@ -105,6 +105,10 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t sw128_chunk(int r, int cc) {
   return static_cast<uint32_t>((cc >> 3) * 16384 + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
 }
+// Same for a tile whose 64-column blocks are `block` bytes apart.
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int cc, uint32_t block) {
+  return static_cast<uint32_t>((cc >> 3) * block + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
+}
 
 // 16-byte shared-memory load / store. The loads carry no memory clobber, so the
 // compiler may hoist the next chunks' loads above this chunk's store (the table and

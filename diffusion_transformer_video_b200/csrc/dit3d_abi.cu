@@ -16,6 +16,7 @@
 #include "../../include/dit3d.h"
 #include "adaln.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_2sm.cuh"
 #include "common.cuh"
 #include "rope3d.cuh"
 
@@ -25,6 +26,7 @@ namespace {
 
 std::mutex g_mu;
 int g_force_timeout = 0;
+int g_attn_variant = 0;  // 0: one CTA per query-tile pair; 1: CTA pairs (head_dim 128)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -202,13 +204,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, H*d] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle.
-bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols) {
+// [rows, H*d] bf16, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
+               uint32_t box_rows = 128) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -235,6 +238,41 @@ int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32
   }
   dim3 grid(n_work, H);
   attn::attn_fwd_kernel<D><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
+  return launch_status();
+}
+
+// head_dim 128 on CTA pairs (cta_group::2): 512 query rows per pair.
+int launch_attn_2sm(const void* q, const void* k, const void* v, int64_t rows, int32_t H,
+                    attn::Params prm, const std::vector<int64_t>& lens, bool dense,
+                    cudaStream_t stream) {
+  constexpr int D = attn2::kD;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, rows, static_cast<int64_t>(H) * D, 128) ||
+      !make_tmap(&tk, k, rows, static_cast<int64_t>(H) * D, attn2::kHalfN) ||
+      !make_tmap(&tv, v, rows, static_cast<int64_t>(H) * D, attn2::kTileN))
+    return DIT_ERR_LAUNCH;
+  int64_t units = 0;
+  if (dense) {
+    prm.pairs_per_dense_seq =
+        static_cast<int32_t>((prm.dense_len + attn2::kPairRows - 1) / attn2::kPairRows);
+    units = static_cast<int64_t>(prm.pairs_per_dense_seq) * prm.n_seq;
+  } else {
+    for (int64_t L : lens) units += (L + attn2::kPairRows - 1) / attn2::kPairRows;
+  }
+  if (units == 0) return DIT_OK;
+  if (2 * units > INT32_MAX) return DIT_ERR_SHAPE;
+  constexpr uint32_t smem = attn2::Smem::kRequest;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(attn2::attn_fwd_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return DIT_ERR_LAUNCH;
+    attr_set[dev] = true;
+  }
+  dim3 grid(static_cast<unsigned>(2 * units), H);
+  attn2::attn_fwd_2sm_kernel<<<grid, attn2::kThreads, smem, stream>>>(tq, tk, tv, prm);
   return launch_status();
 }
 
@@ -402,6 +440,8 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     prm.use_rope = 1;
     if (int s = get_table(rope, t_ext, st, &prm.rope)) return s;
   }
+  if (d == 128 && g_attn_variant == 1)
+    return launch_attn_2sm(q, k, v, rows, H, prm, lens, cu_seqlens_dev == nullptr, st);
   if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
   return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
 }
@@ -428,6 +468,12 @@ void dit_shutdown(void) {
 }
 
 void dit_debug_force_timeout(int enable) { g_force_timeout = enable ? 1 : 0; }
+
+int dit_set_attn_variant(int variant) {
+  if (variant != 0 && variant != 1) return DIT_ERR_SHAPE;
+  g_attn_variant = variant;
+  return DIT_OK;
+}
 
 }  // extern "C"
 
@@ -516,6 +562,8 @@ extern "C" int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v,
     prm.use_rope = 1;
     prm.rope.table = table;
   }
+  if (d == 128 && g_attn_variant == 1)
+    return launch_attn_2sm(q, k, v, rows, H, prm, lens, cu_seqlens_dev == nullptr, st);
   if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
   return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
 }

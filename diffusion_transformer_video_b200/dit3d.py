@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
 # every symbol include/dit3d.h declares
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
-           "dit_debug_force_timeout")
+           "dit_set_attn_variant", "dit_debug_force_timeout")
 
 
 class DitError(RuntimeError):
@@ -71,6 +71,8 @@ def lib():
         L.dit_status_string.restype = ctypes.c_char_p
         L.dit_shutdown.argtypes = []
         L.dit_shutdown.restype = None
+        L.dit_set_attn_variant.argtypes = [ctypes.c_int]
+        L.dit_set_attn_variant.restype = ctypes.c_int
         L.dit_debug_force_timeout.argtypes = [ctypes.c_int]
         L.dit_debug_force_timeout.restype = None
         for name in ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
@@ -184,6 +186,11 @@ def dit_attn_fwd(q, k, v, n_seq=1, cu_seqlens=None, rope: RopeDesc | None = None
                               ctypes.byref(rope) if rope is not None else None, _stream()))
     _keep(cu_dev)
     return (out, lse) if return_lse else out
+
+
+def dit_set_attn_variant(variant: int):
+    """0: single-CTA attention kernel (default); 1: CTA-pair kernel (head_dim 128)."""
+    _check(lib().dit_set_attn_variant(int(variant)))
 
 
 def dit_check_device():

@@ -158,6 +158,14 @@ const char* dit_status_string(int status);
 /* Frees the cached RoPE tables of every device. Safe to call more than once. */
 void dit_shutdown(void);
 
+/* Selects the attention kernel for head_dim 128 (process-wide; head_dim 64 always
+ * uses variant 0). 0 (default): one CTA per 256 query rows of a head on one SM.
+ * 1: CTA pairs on two SMs sharing each tcgen05 MMA (cta_group::2, M = 256): each SM
+ * loads and rotates half of every K tile and loads half of every V tile. Both give the
+ * same results (same rounding steps); variant 0 is faster on the measured workloads.
+ * Returns DIT_ERR_SHAPE for any other value. */
+int dit_set_attn_variant(int variant);
+
 /* Test hook: 1 makes the next attention launches give up their first wait at once
  * (exercising the bounded-wait error path without any hang), 0 restores. */
 void dit_debug_force_timeout(int enable);
