@@ -34,11 +34,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
 UNIT = "TFLOP/s"
-# DRAM bytes of one fused-RoPE attention launch per head, from an ncu capture of the 480P
-# geometry with 16 heads (528 MB / 16; profiles/attn_fwd_fused_rope_480p.md). Heads are
-# independent, so the traffic of the 480P launch is this times its head count. Other
-# workloads have no capture: their traffic is reported as null.
-ATTN_DRAM_BYTES_PER_HEAD_480P = 528.09e6 / 16
+# DRAM bytes per head of one attention launch at the 480P geometry, from an ncu capture
+# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum over 16), keyed by RoPE mode
+# ("prepass" and "none" run the same kernel, without in-kernel RoPE). Heads are
+# independent, so a launch's traffic is this times its head count. None where the
+# current kernel has not been captured; other workloads report null.
+ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": None, "none": None, "fused": None}
 
 
 def _peaks():
@@ -74,6 +75,13 @@ class ClockSampler:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+        # nvidia-smi takes a moment to start: wait (bounded) for its first sample so that
+        # even a short timed region is covered
+        deadline = time.time() + 5.0
+        while self.proc is not None and time.time() < deadline and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
         return self
 
     def __exit__(self, *a):
@@ -188,10 +196,10 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=24, help="oracle sample rows per step")
     ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--rope-mode", default="fused", choices=["fused", "prepass", "none"],
-                    help="fused: RoPE inside the attention kernel (the product path); prepass: "
-                         "dit_rope3d_qk into scratch then attention; none: attention alone "
-                         "(not the workload, a kernel-speed reference)")
+    ap.add_argument("--rope-mode", default="prepass", choices=["prepass", "fused", "none"],
+                    help="prepass: dit_rope3d_qk into scratch, then attention (the product "
+                         "path, fastest); fused: RoPE inside the attention kernel (no scratch); "
+                         "none: attention alone (not the workload, a kernel-speed reference)")
     ap.add_argument("--attn-variant", type=int, default=0, choices=[0, 1],
                     help="0: single-CTA attention kernel; 1: CTA-pair (cta_group::2) kernel")
     ap.add_argument("--heads", type=int, default=0,
@@ -247,29 +255,27 @@ def main():
     if args.rope_mode == "prepass":
         q_rot, k_rot = torch.empty_like(dev["q"]), torch.empty_like(dev["k"])
 
-    def attention(b):
-        if args.rope_mode == "fused":
-            dit3d.dit_attn_fwd(b["q"], b["k"], b["v"], n_seq=w.n_seq, cu_seqlens=cu, rope=desc,
-                               out=o)
-        elif args.rope_mode == "prepass":
-            dit3d.dit_rope3d_qk(b["q"], b["k"], desc, n_seq=w.n_seq, cu_seqlens=cu,
-                                q_out=q_rot, k_out=k_rot)
-            dit3d.dit_attn_fwd(q_rot, k_rot, b["v"], n_seq=w.n_seq, cu_seqlens=cu, out=o)
-        else:
-            dit3d.dit_attn_fwd(b["q"], b["k"], b["v"], n_seq=w.n_seq, cu_seqlens=cu, out=o)
-
     def step(b, ev=None):
         if ev is not None:
             ev[0].record(stream)
         dit3d.dit_adaln_modulate(b["x"], b["gamma"], b["beta"], rpg, out=u)
         if ev is not None:
             ev[1].record(stream)
-        attention(b)
+        if args.rope_mode == "prepass":
+            dit3d.dit_rope3d_qk(b["q"], b["k"], desc, n_seq=w.n_seq, cu_seqlens=cu,
+                                q_out=q_rot, k_out=k_rot)
+            qa, ka = q_rot, k_rot
+        else:
+            qa, ka = b["q"], b["k"]
         if ev is not None:
             ev[2].record(stream)
-        dit3d.dit_gated_residual(b["x"], o.view(rows, D), b["alpha"], rpg, out=out)
+        dit3d.dit_attn_fwd(qa, ka, b["v"], n_seq=w.n_seq, cu_seqlens=cu, out=o,
+                           rope=desc if args.rope_mode == "fused" else None)
         if ev is not None:
             ev[3].record(stream)
+        dit3d.dit_gated_residual(b["x"], o.view(rows, D), b["alpha"], rpg, out=out)
+        if ev is not None:
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step(dev)
@@ -277,7 +283,7 @@ def main():
     dit3d.dit_check_device()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
@@ -292,8 +298,9 @@ def main():
     dit3d.dit_check_device()
     elapsed_ms = t_start.elapsed_time(t_end)
     t_mod = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    t_att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    t_res = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    t_rope = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    t_att = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    t_res = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
     clocks = clk.summary()
 
     # end to end: pinned host inputs -> device, the path, result -> pinned host
@@ -329,6 +336,10 @@ def main():
     res_bytes = 6.0 * rows * D
     mod_gbs = mod_bytes / (t_mod * 1e-3) / 1e9
     res_gbs = res_bytes / (t_res * 1e-3) / 1e9
+    rope_bytes = 8.0 * rows * H * d  # q and k read, rotated q and k written, bf16
+    rope_gbs = rope_bytes / (t_rope * 1e-3) / 1e9 if args.rope_mode == "prepass" else None
+    per_head = ATTN_DRAM_BYTES_PER_HEAD_480P.get(args.rope_mode) if w.name == "480p" else None
+    traffic = per_head * H if per_head is not None and args.attn_variant == 0 else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -353,18 +364,19 @@ def main():
             "roofline": {"bound": "tensor", "achieved": att_tflops,
                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": att_tflops / pk["bf16_tflops_sustained"],
-                         "traffic": (ATTN_DRAM_BYTES_PER_HEAD_480P * H
-                                     if w.name == "480p" and args.rope_mode == "fused" else None),
-                         "attn_variant": ["single CTA", "CTA pair (cta_group::2)"][args.attn_variant],
-                         "kernel": {"fused": "dit_attn_fwd (fused 3D-RoPE)",
-                                    "prepass": "dit_rope3d_qk + dit_attn_fwd",
+                         "traffic": traffic,
+                         "kernel": {"prepass": "dit_attn_fwd (operands rotated by dit_rope3d_qk)",
+                                    "fused": "dit_attn_fwd (fused 3D-RoPE)",
                                     "none": "dit_attn_fwd without RoPE"}[args.rope_mode],
+                         "attn_variant": ["single CTA", "CTA pair (cta_group::2)"][args.attn_variant],
                          "peak_source": f"{pk['source']} sustained bf16 "
                                         f"(burst {pk['bf16_tflops']}: frac "
                                         f"{att_tflops / pk['bf16_tflops']:.3f})"},
             "components": {
                 "adaln_modulate": {"ms": t_mod, "GB/s": mod_gbs, "frac_hbm": mod_gbs / pk["hbm_gbs"],
                                    "bytes": mod_bytes},
+                "rope3d_qk": ({"ms": t_rope, "GB/s": rope_gbs, "frac_hbm": rope_gbs / pk["hbm_gbs"],
+                               "bytes": rope_bytes} if args.rope_mode == "prepass" else None),
                 "attn_fwd": {"ms": t_att, "TFLOP/s": att_tflops, "flops": flops},
                 "gated_residual": {"ms": t_res, "GB/s": res_gbs, "frac_hbm": res_gbs / pk["hbm_gbs"],
                                    "bytes": res_bytes},

@@ -123,6 +123,14 @@ __device__ __forceinline__ float4 lds128f(uint32_t a) {
   asm("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
   return v;
 }
+// Ordered 16-byte load: after every earlier store and never merged with another load
+// of the same address (a chunk re-read after its own rotation was written back).
+__device__ __forceinline__ uint4 lds128_ordered(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a) : "memory");
+  return v;
+}
 __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
@@ -182,9 +190,10 @@ __device__ __forceinline__ void rope_tile_smem(uint32_t tile, int64_t row0, int 
     if (c < 0 || (k && c == cs1)) continue;
     const int a_lo = rope_band_of_pair(rp, 4 * c), a_hi = rope_band_of_pair(rp, 4 * c + 3);
     for (int a = a_lo + 1; a <= a_hi; ++a) {
+      if (rope_band_stride(rp, a) == 0) continue;  // an empty middle band
       const uint32_t e = (a == 1 ? row_h : row_w) + 32u * c;
       const uint32_t ad = tile + sw128_chunk(rt, c);
-      sts128(ad, rope_apply(lds128(ad), lds128f(e), lds128f(e + 16u)));
+      sts128(ad, rope_apply(lds128_ordered(ad), lds128f(e), lds128f(e + 16u)));
     }
   }
 }

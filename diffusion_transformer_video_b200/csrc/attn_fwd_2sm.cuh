@@ -43,6 +43,7 @@ namespace attn2 {
 using attn::ex2;
 using attn::lds128;
 using attn::lds128f;
+using attn::lds128_ordered;
 using attn::Params;
 using attn::rope_apply;
 using attn::sts128;
@@ -123,9 +124,10 @@ __device__ __forceinline__ void rope_row_range(uint32_t tile, uint32_t block, in
     if (c < c_lo || c >= c_lo + NCH || (k && c == cs1)) continue;
     const int a_lo = rope_band_of_pair(rp, 4 * c), a_hi = rope_band_of_pair(rp, 4 * c + 3);
     for (int a = a_lo + 1; a <= a_hi; ++a) {
+      if (rope_band_stride(rp, a) == 0) continue;  // an empty middle band
       const uint32_t e = (a == 1 ? row_h : row_w) + 32u * c;
       const uint32_t ad = tile + sw128_chunk(r, c, block);
-      sts128(ad, rope_apply(lds128(ad), lds128f(e), lds128f(e + 16u)));
+      sts128(ad, rope_apply(lds128_ordered(ad), lds128f(e), lds128f(e + 16u)));
     }
   }
 }

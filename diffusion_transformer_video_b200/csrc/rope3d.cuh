@@ -74,14 +74,21 @@ __device__ __forceinline__ void rope_rotate4(float (&x)[8], float4 f01, float4 f
   rope_rotate_couple(x[4], x[5], x[6], x[7], f23);
 }
 
+// Width (in float2 entries per position) of band a's table section; 0 for an empty band.
+__device__ __forceinline__ int rope_band_stride(const RopeParams& rp, int a) {
+  return a == 0 ? rp.str0 : (a == 1 ? rp.str1 : rp.str2);
+}
+
 // Rotate chunk c (pairs 4c .. 4c+3) of one row at position (t, h, w). `tab` is the
-// table (in global or shared memory, generic address).
+// table (in global or shared memory, generic address). The bands are applied in
+// order; an empty band between two others (d_h = 0) has no section and is skipped.
 __device__ __forceinline__ uint4 rope_chunk(const RopeParams& rp, const float2* tab, uint4 v, int c,
                                             int t, int h, int w) {
   float x[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
                 bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
   const int a_lo = rope_band_of_pair(rp, 4 * c), a_hi = rope_band_of_pair(rp, 4 * c + 3);
   for (int a = a_lo; a <= a_hi; ++a) {
+    if (rope_band_stride(rp, a) == 0) continue;
     const int pos = a == 0 ? t : (a == 1 ? h : w);
     const float4* e = reinterpret_cast<const float4*>(tab + rope_entry(rp, a, pos, c));
     rope_rotate4(x, e[0], e[1]);
@@ -102,29 +109,81 @@ __device__ __forceinline__ int64_t seq_start_of_row(const int32_t* __restrict__ 
   return __ldg(cu + lo);
 }
 
-// Standalone RoPE: one warp per token row; lane l handles chunk l % (D_HEAD/8) of
-// every head of q and of k, with the same per-chunk procedure as the attention
-// kernel (so both produce the same bits).
+// The rotation of one chunk by up to three bands whose table entries are already in
+// registers (nb of them, in band order): the arithmetic of rope_chunk.
+__device__ __forceinline__ uint4 rope_chunk_reg(uint4 v, int nb, const float4 (&f)[3][2]) {
+  float x[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
+                bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+  rope_rotate4(x, f[0][0], f[0][1]);
+  if (nb > 1) rope_rotate4(x, f[1][0], f[1][1]);
+  if (nb > 2) rope_rotate4(x, f[2][0], f[2][1]);
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
+}
+
+// Standalone RoPE, an HBM stream: one warp per token row. Lane l always handles
+// chunk l % (D_HEAD/8) of a head, so the row's table entries for that chunk are read
+// once into registers and reused for every head of q and of k; the head loop keeps
+// kUnroll 16-byte loads of q and of k in flight per lane before rotating and
+// storing them. Same per-chunk arithmetic as rope_chunk (and the attention kernel),
+// so all produce the same bits. In place (q_out == q_in) is safe: every element is
+// read and written by the same thread.
 template <int D_HEAD>
 __global__ void __launch_bounds__(256)
 rope3d_qk_kernel(const uint4* q_in, const uint4* k_in, uint4* q_out, uint4* k_out, int64_t rows,
                  int32_t H, const int32_t* __restrict__ cu, int32_t n_seq, int64_t dense_len,
                  RopeParams rp) {
-  static_assert(32 % (D_HEAD / 8) == 0, "lane-fixed chunks need D_HEAD/8 to divide 32");
+  constexpr int kCpr = D_HEAD / 8;  // 16-byte chunks per head
+  constexpr int kUnroll = 4;
+  static_assert(32 % kCpr == 0, "lane-fixed chunks need D_HEAD/8 to divide 32");
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int64_t j = row - seq_start_of_row(cu, n_seq, row, dense_len);
   int t, h, w;
   token_pos(j, rp.grid_h, rp.grid_w, t, h, w);
-  const int cc = lane % (D_HEAD / 8);
-  const int nchunk = H * (D_HEAD / 8);
+  const int cc = lane % kCpr;
+  const float4 one = make_float4(1.f, 1.f, 0.f, 0.f);  // identity (cos 1, sin 0)
+  float4 f[3][2] = {{one, one}, {one, one}, {one, one}};
+  int nb = 0;
+  const int a_lo = rope_band_of_pair(rp, 4 * cc), a_hi = rope_band_of_pair(rp, 4 * cc + 3);
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    if (a < a_lo || a > a_hi || rope_band_stride(rp, a) == 0) continue;
+    const int pos = a == 0 ? t : (a == 1 ? h : w);
+    const float4* e = reinterpret_cast<const float4*>(rp.table + rope_entry(rp, a, pos, cc));
+    const float4 e0 = __ldg(e), e1 = __ldg(e + 1);
+    // nb is 0, 1 or 2 here; selects keep f in registers
+    f[0][0] = nb == 0 ? e0 : f[0][0];
+    f[0][1] = nb == 0 ? e1 : f[0][1];
+    f[1][0] = nb == 1 ? e0 : f[1][0];
+    f[1][1] = nb == 1 ? e1 : f[1][1];
+    f[2][0] = nb == 2 ? e0 : f[2][0];
+    f[2][1] = nb == 2 ? e1 : f[2][1];
+    ++nb;
+  }
+  const int nchunk = H * kCpr;
   const int64_t base = row * nchunk;
-  for (int c = lane; c < nchunk; c += 32)
-    q_out[base + c] = rope_chunk(rp, rp.table, q_in[base + c], cc, t, h, w);
-  if (k_in != nullptr)
-    for (int c = lane; c < nchunk; c += 32)
-      k_out[base + c] = rope_chunk(rp, rp.table, k_in[base + c], cc, t, h, w);
+  const bool has_k = k_in != nullptr;
+  for (int c0 = lane; c0 < nchunk; c0 += 32 * kUnroll) {
+    uint4 vq[kUnroll], vk[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nchunk) {
+        vq[u] = q_in[base + c];
+        if (has_k) vk[u] = k_in[base + c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nchunk) {
+        q_out[base + c] = rope_chunk_reg(vq[u], nb, f);
+        if (has_k) k_out[base + c] = rope_chunk_reg(vk[u], nb, f);
+      }
+    }
+  }
 }
 
 }  // namespace dit3d

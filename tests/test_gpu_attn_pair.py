@@ -31,11 +31,15 @@ def test_pair_attn_parity(pair_variant, lens):
     np.testing.assert_allclose(lse, ref_lse, atol=2e-2)
 
 
-@pytest.mark.parametrize("gh,gw,frames", [(3, 5, [9, 2, 20]), (16, 16, [1]), (30, 52, [3])])
-def test_pair_fused_rope_parity(pair_variant, gh, gw, frames):
+@pytest.mark.parametrize("gh,gw,frames,bands", [(3, 5, [9, 2, 20], (44, 42, 42)),
+                                                (16, 16, [1], (44, 42, 42)),
+                                                (30, 52, [3], (44, 42, 42)),
+                                                (3, 4, [11, 2], (6, 0, 122)),
+                                                (3, 3, [30], (2, 4, 122))])
+def test_pair_fused_rope_parity(pair_variant, gh, gw, frames, bands):
     lens = [f * gh * gw for f in frames]
     q, k, v, cu = _attn_case(lens, 2, 128, seed=23)
-    rope_kw = dict(grid_h=gh, grid_w=gw, bands=(44, 42, 42), base=10000.0, offsets=(0, 1, 2))
+    rope_kw = dict(grid_h=gh, grid_w=gw, bands=bands, base=10000.0, offsets=(0, 1, 2))
     o, lse = _run_attn(q, k, v, cu, rope_kw)
     ref_o, ref_lse = oracle.attn_fwd(f64(q), f64(k), f64(v), cu, rope=rope_kw)
     check_attention(o, ref_o, "pair fused rope")

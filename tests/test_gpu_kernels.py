@@ -65,11 +65,17 @@ def _rope_ref(v_bits, cu, grid_h, grid_w, bands, base=10000.0, offsets=(0, 0, 0)
     return oracle.rope3d(f64(v_bits), cu, grid_h, grid_w, bands, base, offsets)
 
 
-@pytest.mark.parametrize("d,bands,gh,gw,frames", [(64, (16, 24, 24), 4, 4, [4]),
-                                                   (128, (44, 42, 42), 3, 5, [2, 7, 1]),
-                                                   (128, (32, 48, 48), 8, 8, [1, 1])])
-def test_rope3d_parity(d, bands, gh, gw, frames):
-    H = 3
+@pytest.mark.parametrize("d,bands,gh,gw,frames,H", [
+    (64, (16, 24, 24), 4, 4, [4], 3),
+    (128, (44, 42, 42), 3, 5, [2, 7, 1], 3),
+    (128, (32, 48, 48), 8, 8, [1, 1], 3),
+    (128, (44, 42, 42), 30, 52, [2], 40),   # the 480P row width: 40 heads
+    (128, (6, 0, 122), 3, 4, [2, 3], 5),    # empty middle band inside a chunk
+    (128, (0, 64, 64), 2, 3, [3], 2),       # empty first band
+    (64, (20, 44, 0), 3, 3, [2], 7),        # empty last band
+    (64, (2, 2, 60), 2, 2, [5], 1),         # one chunk turned by all three bands
+])
+def test_rope3d_parity(d, bands, gh, gw, frames, H):
     lens = [f * gh * gw for f in frames]
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     rows = int(cu[-1])
@@ -149,7 +155,10 @@ def test_attn_varlen_parity(lens):
 
 @pytest.mark.parametrize("d,bands,gh,gw,frames", [(64, (16, 24, 24), 4, 4, [4]),
                                                    (128, (44, 42, 42), 3, 5, [9, 2, 20]),
-                                                   (128, (32, 48, 48), 16, 16, [1])])
+                                                   (128, (32, 48, 48), 16, 16, [1]),
+                                                   (128, (6, 0, 122), 3, 4, [11, 2]),
+                                                   (128, (2, 4, 122), 3, 3, [30]),
+                                                   (64, (2, 2, 60), 4, 4, [9])])
 def test_attn_fused_rope_parity(d, bands, gh, gw, frames):
     lens = [f * gh * gw for f in frames]
     q, k, v, cu = _attn_case(lens, 2, d, seed=11)
@@ -160,11 +169,13 @@ def test_attn_fused_rope_parity(d, bands, gh, gw, frames):
     np.testing.assert_allclose(lse, ref_lse, atol=2e-2)
 
 
-def test_attn_fused_rope_equals_rope_then_attn():
+@pytest.mark.parametrize("d,bands", [(128, (44, 42, 42)), (128, (6, 0, 122)), (128, (2, 4, 122)),
+                                     (64, (2, 2, 60))])
+def test_attn_fused_rope_equals_rope_then_attn(d, bands):
     gh, gw, frames = 5, 6, [7, 3]
     lens = [f * gh * gw for f in frames]
-    q, k, v, cu = _attn_case(lens, 3, 128, seed=5)
-    desc = dit3d.rope_desc(gh, gw, (44, 42, 42))
+    q, k, v, cu = _attn_case(lens, 3, d, seed=5)
+    desc = dit3d.rope_desc(gh, gw, bands, 10000.0, (2, 1, 3))
     qr, kr = dit3d.dit_rope3d_qk(to_dev(q), to_dev(k), desc, cu_seqlens=cu)
     o_two = dit3d.dit_attn_fwd(qr, kr, to_dev(v), cu_seqlens=cu)
     o_fused = dit3d.dit_attn_fwd(to_dev(q), to_dev(k), to_dev(v), cu_seqlens=cu, rope=desc)
