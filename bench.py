@@ -303,6 +303,23 @@ def main():
     t_res = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
     clocks = clk.summary()
 
+    # the sampler's Euler step (x += dt_frame * u), timed on its own: not part of the step
+    frame = w.grid_h * w.grid_w
+    dt_dev = torch.from_numpy(
+        np.random.default_rng([args.seed, 99]).uniform(0.0, 0.1, rows // frame).astype(np.float32)).cuda()
+    x_next = torch.empty_like(dev["x"])
+    u_vel = o.view(rows, D)
+    for _ in range(3):
+        dit3d.dit_flow_euler_step(dev["x"], u_vel, dt_dev, frame, out=x_next)
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ee:
+        a.record(stream)
+        dit3d.dit_flow_euler_step(dev["x"], u_vel, dt_dev, frame, out=x_next)
+        b.record(stream)
+    torch.cuda.synchronize()
+    dit3d.dit_check_device()
+    t_euler = statistics.mean(a.elapsed_time(b) for a, b in ee)
+
     # end to end: pinned host inputs -> device, the path, result -> pinned host
     e2e_keys = ("x", "q", "k", "v", "gamma", "beta", "alpha")
     dev2 = {k: torch.empty_like(dev[k]) for k in e2e_keys}
@@ -380,6 +397,10 @@ def main():
                 "attn_fwd": {"ms": t_att, "TFLOP/s": att_tflops, "flops": flops},
                 "gated_residual": {"ms": t_res, "GB/s": res_gbs, "frac_hbm": res_gbs / pk["hbm_gbs"],
                                    "bytes": res_bytes},
+                "flow_euler_step": {"ms": t_euler, "GB/s": res_bytes / (t_euler * 1e-3) / 1e9,
+                                    "frac_hbm": res_bytes / (t_euler * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                    "bytes": res_bytes, "in_step": False,
+                                    "note": "sampler update x += dt_frame * u, timed separately"},
             },
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -18,6 +18,7 @@
 #include "attn_fwd.cuh"
 #include "attn_fwd_2sm.cuh"
 #include "common.cuh"
+#include "flow_euler.cuh"
 #include "rope3d.cuh"
 
 using namespace dit3d;
@@ -292,6 +293,14 @@ void launch_residual(const void* x, const void* y, const void* a, void* o, int64
       static_cast<const __nv_bfloat16*>(a), static_cast<__nv_bfloat16*>(o), D, rpg);
 }
 
+template <int NV>
+void launch_euler(const void* x, const void* u, const float* dt, void* o, int64_t rows, int32_t D,
+                  int64_t rpg, cudaStream_t st) {
+  flow_euler_kernel<NV><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(u), dt,
+      static_cast<__nv_bfloat16*>(o), D, rpg);
+}
+
 }  // namespace
 
 extern "C" {
@@ -366,6 +375,33 @@ int dit_gated_residual(const void* x, const void* y, const void* alpha, void* ou
           static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y),
           static_cast<const __nv_bfloat16*>(alpha), static_cast<__nv_bfloat16*>(out), D,
           rows_per_group);
+  }
+  return launch_status();
+}
+
+int dit_flow_euler_step(const void* x, const void* u, const float* dt, void* out, int64_t rows,
+                        int32_t D, int64_t rows_per_group, void* stream) {
+  if (!x || !u || !dt || !out) return DIT_ERR_NULL;
+  if (int s = check_rows_groups(rows, D, rows_per_group)) return s;
+  if (!aligned16(x) || !aligned16(u) || !aligned16(out) || (reinterpret_cast<uintptr_t>(dt) & 3u))
+    return DIT_ERR_ALIGN;
+  if (int s = check_device()) return s;
+  if (rows == 0) return DIT_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  const int nv = (D / 8 + kRowThreads - 1) / kRowThreads;
+  switch (nv) {
+    case 1: launch_euler<1>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 2: launch_euler<2>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 3: launch_euler<3>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 4: launch_euler<4>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 5: launch_euler<5>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 6: launch_euler<6>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 7: launch_euler<7>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    case 8: launch_euler<8>(x, u, dt, out, rows, D, rows_per_group, st); break;
+    default:
+      flow_euler_wide_kernel<<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(u), dt,
+          static_cast<__nv_bfloat16*>(out), D, rows_per_group);
   }
   return launch_status();
 }

@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
                 7: "DIT_ERR_TIMEOUT", 8: "DIT_ERR_ALLOC", 9: "DIT_ERR_SCRATCH"}
 
 # every symbol include/dit3d.h declares
-EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
+EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_rope3d_qk",
+           "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout")
 
@@ -59,6 +60,7 @@ def lib():
         P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
         L.dit_adaln_modulate.argtypes = [P, P, P, P, i64, i32, i64, f32, f32, P]
         L.dit_gated_residual.argtypes = [P, P, P, P, i64, i32, i64, P]
+        L.dit_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64, P]
         L.dit_rope3d_qk.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
                                     ctypes.POINTER(RopeDesc), P]
         L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
@@ -148,6 +150,24 @@ def dit_gated_residual(x, y, alpha, rows_per_group, out=None):
     rows, D = x.shape[0], x.shape[-1]
     _check(lib().dit_gated_residual(_ptr(x), _ptr(y), _ptr(alpha), _ptr(out), rows, D,
                                     int(rows_per_group), _stream()))
+    return out
+
+
+def dit_flow_euler_step(x, u, dt, rows_per_group, out=None):
+    """out = x + dt[g] * u for the rows of frame g (x, u [rows, D] bf16; dt [G] fp32 on the
+    device). out=x updates the latent in place."""
+    _bf16(x, "x")
+    _bf16(u, "u")
+    if not (isinstance(dt, torch.Tensor) and dt.dtype == torch.float32 and dt.is_cuda
+            and dt.is_contiguous()):
+        raise TypeError("dt must be a contiguous float32 CUDA tensor")
+    out = torch.empty_like(x) if out is None else out
+    _bf16(out, "out")
+    rows, D = x.shape[0], x.shape[-1]
+    if rows == 0:
+        return out
+    _check(lib().dit_flow_euler_step(_ptr(x), _ptr(u), _ptr(dt), _ptr(out), rows, D,
+                                     int(rows_per_group), _stream()))
     return out
 
 

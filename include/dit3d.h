@@ -6,6 +6,7 @@
  *   q,k = R3D(t, h, w) q,  R3D(t, h, w) k                     dit_rope3d_qk
  *   o   = softmax(q_rot k_rot^T / sqrt(d_head)) v             dit_attn_fwd
  *   out = x + alpha_g * y                                     dit_gated_residual
+ *   x  += dt_frame * u   (sampler step, not in the block)       dit_flow_euler_step
  *
  * Formulas: "DiT, Flow Matching e 3D Attention: A Engenharia de Video com IA",
  * sections "A ruptura da U-Net" (adaLN-Zero) and "3D-RoPE e atencao
@@ -89,6 +90,20 @@ int dit_adaln_modulate(const void* x, const void* gamma, const void* beta, void*
  * Errors: as dit_adaln_modulate. */
 int dit_gated_residual(const void* x, const void* y, const void* alpha, void* out,
                        int64_t rows, int32_t D, int64_t rows_per_group, void* stream);
+
+/* One Euler step of the rectified-flow sampler with per-frame local times (DiT
+ * page, section "Flow Matching e Rectified Flow": straight path x_t = (1-t) x_0 +
+ * t x_1, velocity u, 10-25 Euler or midpoint steps; "Flowception: Temporally
+ * Expansive Flow Matching for Video Generation", section "Metodologia", interleaved
+ * time schedule: each frame i has its own local time t_i):
+ *   out[r, c] = x[r, c] + dt[g] * u[r, c],   g = r / rows_per_group
+ * with dt[g] = t_g' - t_g the step of frame g (rows_per_group = tokens per frame).
+ * fp32 FMA, one bf16 rounding; dt[g] == 0 returns x[r, :] bit for bit.
+ *   x, u, out : [rows, D] bf16 (out may alias x: the in-place sampler update)
+ *   dt        : [rows / rows_per_group] fp32, device memory, 4-byte aligned
+ * Errors: as dit_adaln_modulate; DIT_ERR_NULL for a null pointer. */
+int dit_flow_euler_step(const void* x, const void* u, const float* dt, void* out, int64_t rows,
+                        int32_t D, int64_t rows_per_group, void* stream);
 
 /* Standalone 3D-RoPE of q and k (DiT page, "3D-RoPE e atencao espaco-temporal"),
  * fp32 rotation of bf16 data, the same rotation for every head.

@@ -9,6 +9,10 @@ Each wrapper cites the passage it restates:
 
 * ``adaln_modulate`` / ``gated_residual`` -- "DiT, Flow Matching e 3D Attention",
   section "A ruptura da U-Net" (adaLN-Zero).
+* ``flow_euler_step`` -- same page, section "Flow Matching e Rectified Flow"
+  (Euler sampler on the straight path), with the per-frame local times of
+  "Flowception: Temporally Expansive Flow Matching for Video Generation",
+  section "Metodologia".
 * ``rope3d`` -- same page, section "3D-RoPE e atencao espaco-temporal".
 * ``attn_fwd`` -- same section, and "Por que e absurdamente dificil gerar um
   filme inteiro usando IA", section "Matematica por tras".
@@ -49,11 +53,12 @@ def _load():
         i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
         lib.oracle_adaln_modulate.argtypes = [P, P, P, P, i64, i32, i64, f64, f64]
         lib.oracle_gated_residual.argtypes = [P, P, P, P, i64, i32, i64]
+        lib.oracle_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64]
         lib.oracle_rope3d.argtypes = [P, P, i64, i32, i32, P, i32, i32, i32, i32, i32, i32, f64,
                                       i32, i32, i32]
         lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, P, i32, f64, P, i64]
         for f in (lib.oracle_adaln_modulate, lib.oracle_gated_residual, lib.oracle_rope3d,
-                  lib.oracle_attn_fwd):
+                  lib.oracle_attn_fwd, lib.oracle_flow_euler_step):
             f.restype = None
         _lib = lib
     return _lib
@@ -99,6 +104,17 @@ def gated_residual(x, y, alpha, rows_per_group: int) -> np.ndarray:
     out = np.empty_like(x)
     _load().oracle_gated_residual(_ptr(x), _ptr(y), _ptr(alpha), _ptr(out), rows, D,
                                   rows_per_group)
+    return out
+
+
+def flow_euler_step(x, u, dt, rows_per_group: int) -> np.ndarray:
+    """out = x + dt[g] * u for the rows of frame g, fp64. x, u: [rows, D]; dt: [G]."""
+    x, u, dt = _f64(x), _f64(u), _f64(dt)
+    rows, D = x.shape
+    assert u.shape == x.shape and dt.shape == (rows // rows_per_group,)
+    out = np.empty_like(x)
+    _load().oracle_flow_euler_step(_ptr(x), _ptr(u), _ptr(dt), _ptr(out), rows, D,
+                                   rows_per_group)
     return out
 
 

@@ -88,6 +88,22 @@ void oracle_gated_residual(const double* x, const double* y, const double* alpha
 }
 
 /*
+ * One explicit Euler step of the rectified-flow ODE dx/dt = u (page 2, "Flow
+ * Matching e Rectified Flow": straight path x_t = (1-t) x_0 + t x_1 whose velocity
+ * is x_1 - x_0; Euler sampler) with per-frame local times (page 3, Flowception,
+ * "Metodologia": frame i has its own time t_i, so its step is dt_i = t_i' - t_i):
+ *   out[r, c] = x[r, c] + dt[r / rows_per_group] * u[r, c].
+ */
+void oracle_flow_euler_step(const double* x, const double* u, const double* dt, double* out,
+                            int64_t rows, int32_t D, int64_t rows_per_group) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    const double h = dt[r / rows_per_group];
+    for (int32_t c = 0; c < D; ++c) out[r * D + c] = x[r * D + c] + h * u[r * D + c];
+  }
+}
+
+/*
  * 3D rotary position embedding (page 2, "3D-RoPE e atencao espaco-temporal").
  * The head dimension is cut into three contiguous bands [t | h | w] of widths
  * d_t, d_h, d_w (each even, summing to d). Within band a, the pair

@@ -59,6 +59,41 @@ def test_gated_residual_alpha_zero_is_bitwise_identity():
     assert torch.equal(out.view(torch.int16), xt.view(torch.int16))
 
 
+# ----------------------------------------------------------------------------- Euler step
+
+@pytest.mark.parametrize("rows,D,rpg", [(1, 8, 1), (60, 136, 12), (64, 3072, 16), (21, 5120, 3),
+                                        (6, 9216, 2), (0, 64, 1)])
+def test_flow_euler_step_parity(rows, D, rpg):
+    x, u = bits((rows, D)), bits((rows, D))
+    G = max(rows // rpg, 1)
+    dt = RNG.uniform(-0.2, 0.2, G).astype(np.float32)
+    dt[0] = 0.0  # a frame already at its final time
+    out = dit3d.dit_flow_euler_step(to_dev(x), to_dev(u), torch.from_numpy(dt).cuda(), rpg)
+    dit3d.dit_check_device()
+    if rows == 0:
+        return
+    got, ref = from_dev(out), oracle.flow_euler_step(f64(x), f64(u), dt.astype(np.float64), rpg)
+    check_modulation(got, ref, "euler")
+    # zero step: the frame's rows keep their bits
+    np.testing.assert_array_equal(out[:rpg].view(torch.int16).cpu().numpy(),
+                                  x[:rpg].view(np.int16))
+
+
+def test_flow_euler_step_in_place_and_errors():
+    rows, D, rpg = 48, 1024, 16
+    x, u = bits((rows, D)), bits((rows, D))
+    dt = torch.tensor([0.1, -0.3, 0.05], dtype=torch.float32, device="cuda")
+    xa = to_dev(x)
+    ref = dit3d.dit_flow_euler_step(xa, to_dev(u), dt, rpg)
+    dit3d.dit_flow_euler_step(xa, to_dev(u), dt, rpg, out=xa)
+    assert torch.equal(xa, ref)
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_flow_euler_step(xa, to_dev(u), dt, 5)  # 48 rows do not split into groups of 5
+    assert e.value.status == 2
+    L = dit3d.lib()
+    assert L.dit_flow_euler_step(None, None, None, None, rows, D, rpg, None) == 1
+
+
 # ----------------------------------------------------------------------------- RoPE
 
 def _rope_ref(v_bits, cu, grid_h, grid_w, bands, base=10000.0, offsets=(0, 0, 0)):

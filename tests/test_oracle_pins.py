@@ -151,6 +151,42 @@ def _rope(v, cu, gh, gw, bands, base=10000.0, offsets=(0, 0, 0)):
     return oracle.rope3d(v, cu, gh, gw, bands, base, offsets)
 
 
+# ----------------------------------------------------------------------------- Euler step
+# DiT page, "Flow Matching e Rectified Flow": on the straight path
+# x_t = (1 - t) x_0 + t x_1 the velocity is the constant x_1 - x_0, so one Euler step of
+# any size lands exactly on the path; Flowception, "Metodologia": frames keep their own
+# local times, so each frame moves along its own path by its own step.
+
+def test_euler_step_is_exact_on_the_straight_path():
+    rng = np.random.default_rng(7)
+    G, rpg, D = 5, 6, 16
+    x0 = rng.standard_normal((G * rpg, D))
+    x1 = rng.standard_normal((G * rpg, D))
+    t = rng.uniform(0.0, 0.9, G)          # local time of each frame
+    t_next = np.minimum(t + rng.uniform(0.01, 0.3, G), 1.0)
+    tr, tr_next = np.repeat(t, rpg)[:, None], np.repeat(t_next, rpg)[:, None]
+    x_t = (1 - tr) * x0 + tr * x1
+    out = oracle.flow_euler_step(x_t, x1 - x0, t_next - t, rpg)
+    np.testing.assert_allclose(out, (1 - tr_next) * x0 + tr_next * x1, rtol=0, atol=1e-12)
+
+
+def test_euler_frames_use_their_own_step():
+    # frame g gets step dt[g]: a constant velocity of ones moves frame g by exactly dt[g]
+    dt = np.array([0.0, 0.5, -0.25, 2.0])
+    x = np.zeros((8, 4))
+    out = oracle.flow_euler_step(x, np.ones_like(x), dt, 2)
+    np.testing.assert_array_equal(out[:, 0], np.repeat(dt, 2))
+
+
+def test_euler_zero_step_is_identity_and_steps_compose():
+    rng = np.random.default_rng(8)
+    x, u = rng.standard_normal((6, 8)), rng.standard_normal((6, 8))
+    np.testing.assert_array_equal(oracle.flow_euler_step(x, u, np.zeros(3), 2), x)
+    a, b = np.array([0.125, 0.25, 0.5]), np.array([0.25, 0.5, 0.125])
+    two = oracle.flow_euler_step(oracle.flow_euler_step(x, u, a, 2), u, b, 2)
+    np.testing.assert_allclose(two, oracle.flow_euler_step(x, u, a + b, 2), atol=1e-14)
+
+
 def test_rope_preserves_norm():
     # Orthogonal rotations (DiT page, 3D-RoPE section): |R q| = |q| per head.
     gh, gw, T, H, d = 3, 5, 4, 3, 64
