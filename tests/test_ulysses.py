@@ -1,0 +1,115 @@
+"""Ulysses sequence parallelism (DiT page, "Engenharia de inferencia e paralelismo
+de contexto: Ulysses, Ring Attention e FP8") on CPU gloo ranks: the two all-to-all
+exchanges regroup tokens and heads exactly, and the whole flow -- exchange, 3D-RoPE
+on the full sequence, per-head attention, exchange back -- equals attention of the
+unsplit sequence. The attention here is the fp64 oracle (test infrastructure); on
+GPUs the same exchanges feed dit_rope3d_qk and dit_attn_fwd."""
+import itertools
+import json
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from diffusion_transformer_video_b200 import ulysses
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "token_grid.json")
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _full(N, H, d, seed):
+    g = np.random.default_rng(seed)
+    return [g.standard_normal((N, H, d)) for _ in range(3)]
+
+
+def _worker(rank, world, port, q, N, H, d, grid):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        n_loc, h_loc = ulysses.ulysses_shapes(N, H, world)
+        Q, K, V = _full(N, H, d, 5)
+        mine = slice(rank * n_loc, (rank + 1) * n_loc)
+        heads = slice(rank * h_loc, (rank + 1) * h_loc)
+        # exchange 1: this rank's tokens -> all tokens of this rank's heads
+        qh = ulysses.seq_to_head(torch.from_numpy(Q[mine].copy()))
+        kh = ulysses.seq_to_head(torch.from_numpy(K[mine].copy()))
+        vh = ulysses.seq_to_head(torch.from_numpy(V[mine].copy()))
+        exact = bool(np.array_equal(qh.numpy(), Q[:, heads]))
+        # round trip
+        back = ulysses.head_to_seq(qh)
+        round_trip = bool(np.array_equal(back.numpy(), Q[mine]))
+        # whole flow: RoPE on the full sequence (global positions), attention per head
+        rope = dict(grid_h=grid[0], grid_w=grid[1], bands=(d // 4, d // 4 + d // 8, d // 2 - d // 8),
+                    base=10000.0, offsets=(0, 0, 0))
+        cu = np.array([0, N], np.int32)
+        qr = oracle.rope3d(qh.numpy(), cu, rope["grid_h"], rope["grid_w"], rope["bands"])
+        kr = oracle.rope3d(kh.numpy(), cu, rope["grid_h"], rope["grid_w"], rope["bands"])
+        oh, _ = oracle.attn_fwd(qr, kr, vh.numpy(), cu)
+        o_loc = ulysses.head_to_seq(torch.from_numpy(np.ascontiguousarray(oh))).numpy()
+        ref, _ = oracle.attn_fwd(Q, K, V, cu, qrows=np.arange(mine.start, mine.stop), rope=rope)
+        err = float(np.abs(o_loc - ref).max())
+        q.put((rank, exact, round_trip, err))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_exchanges_and_attention_equal_the_unsplit_sequence(world):
+    N, H, d, grid = 96, 8, 16, (4, 6)       # 4 frames of a 4x6 patch grid
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, N, H, d, grid))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, exact, round_trip, err in res:
+        assert exact, f"rank {rank}: seq_to_head is not the head slice of the full tensor"
+        assert round_trip, f"rank {rank}: head_to_seq does not invert seq_to_head"
+        assert err < 1e-12, f"rank {rank}: split attention differs from the whole by {err}"
+
+
+def test_ulysses_shapes_match_the_pages_example():
+    g = json.load(open(GOLDEN))
+    n, h = ulysses.ulysses_shapes(g["tokens"], g["ulysses"]["heads"], g["ulysses"]["gpus"])
+    assert (n, h) == (g["ulysses"]["tokens_per_gpu"], g["ulysses"]["heads_per_gpu"])
+    with pytest.raises(ValueError):
+        ulysses.ulysses_shapes(108000, 24, 7)
+
+
+def _makespan(lengths, parts):
+    return max(sum(int(lengths[i]) ** 2 for i in p) for p in parts)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_lpt_assign_is_a_partition_within_four_thirds_of_optimal(seed):
+    rng = np.random.default_rng(seed)
+    lengths = rng.integers(3, 22, 7) * 1560
+    world = 3
+    parts = ulysses.lpt_assign(lengths, world)
+    assert sorted(i for p in parts for i in p) == list(range(len(lengths)))
+    best = min(_makespan(lengths, [[i for i in range(len(lengths)) if a[i] == r] for r in range(world)])
+               for a in itertools.product(range(world), repeat=len(lengths)))
+    assert _makespan(lengths, parts) <= 4 / 3 * best + 1e-9   # Graham's LPT bound
+    assert parts == ulysses.lpt_assign(list(lengths), world)  # deterministic
+
+
+def test_lpt_assign_small_cases():
+    assert ulysses.lpt_assign([5, 4, 3, 3], 2) == [[0, 3], [1, 2]]
+    assert ulysses.lpt_assign([1, 1, 1], 4) == [[0], [1], [2], []]
