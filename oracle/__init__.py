@@ -13,6 +13,8 @@ Each wrapper cites the passage it restates:
   (Euler sampler on the straight path), with the per-frame local times of
   "Flowception: Temporally Expansive Flow Matching for Video Generation",
   section "Metodologia".
+* ``linear`` -- "Por que e absurdamente dificil gerar um filme inteiro usando IA",
+  section "Matematica por tras" (Y = X W), with the DiT page's MLP and gates.
 * ``rope3d`` -- same page, section "3D-RoPE e atencao espaco-temporal".
 * ``attn_fwd`` -- same section, and "Por que e absurdamente dificil gerar um
   filme inteiro usando IA", section "Matematica por tras".
@@ -54,11 +56,12 @@ def _load():
         lib.oracle_adaln_modulate.argtypes = [P, P, P, P, i64, i32, i64, f64, f64]
         lib.oracle_gated_residual.argtypes = [P, P, P, P, i64, i32, i64]
         lib.oracle_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64]
+        lib.oracle_linear.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64]
         lib.oracle_rope3d.argtypes = [P, P, i64, i32, i32, P, i32, i32, i32, i32, i32, i32, f64,
                                       i32, i32, i32]
         lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, P, i32, f64, P, i64]
         for f in (lib.oracle_adaln_modulate, lib.oracle_gated_residual, lib.oracle_rope3d,
-                  lib.oracle_attn_fwd, lib.oracle_flow_euler_step):
+                  lib.oracle_attn_fwd, lib.oracle_flow_euler_step, lib.oracle_linear):
             f.restype = None
         _lib = lib
     return _lib
@@ -115,6 +118,26 @@ def flow_euler_step(x, u, dt, rows_per_group: int) -> np.ndarray:
     out = np.empty_like(x)
     _load().oracle_flow_euler_step(_ptr(x), _ptr(u), _ptr(dt), _ptr(out), rows, D,
                                    rows_per_group)
+    return out
+
+
+def linear(x, w, bias=None, act: int = 0, res=None, alpha=None,
+           rows_per_group: int = 1) -> np.ndarray:
+    """y = x w^T (+ bias), GELU (tanh form) if act == 1, then res + alpha_g * y when res
+    is given; fp64. x: [M, K]; w: [N, K]; bias: [N]; res: [M, N]; alpha: [G, N]."""
+    x, w = _f64(x), _f64(w)
+    M, K = x.shape
+    N = w.shape[0]
+    assert w.shape == (N, K)
+    b = None if bias is None else _f64(bias)
+    r = None if res is None else _f64(res)
+    a = None if alpha is None else _f64(alpha)
+    if r is not None:
+        assert r.shape == (M, N) and a is not None and a.shape == (M // rows_per_group, N)
+    out = np.empty((M, N))
+    _load().oracle_linear(_ptr(x), _ptr(w), None if b is None else _ptr(b), _ptr(out), M, N, K,
+                          int(act), None if r is None else _ptr(r), None if a is None else _ptr(a),
+                          rows_per_group)
     return out
 
 

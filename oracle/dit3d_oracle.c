@@ -104,6 +104,35 @@ void oracle_flow_euler_step(const double* x, const double* u, const double* dt, 
 }
 
 /*
+ * Linear layer of the block (page 1, "Matematica por tras": Y = X W, cost
+ * O(n d m); page 2, "A ruptura da U-Net": the attention output projection and the
+ * MLP inside the adaLN-Zero residuals):
+ *   y[m, n] = sum_k x[m, k] w[n, k] + bias[n]          (w in [out, in] layout)
+ *   y       = gelu(y) if act == 1, with the tanh form
+ *             gelu(y) = y/2 (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3)))
+ *   out     = y, or res + alpha[g, n] * y (g = m / rows_per_group) when res is given.
+ * Readings (the pages name only "MLP" and the gates): GELU in its tanh form, a
+ * bias per output column, the gate applied after the activation.
+ * bias, res, alpha may be NULL (no bias; plain output).
+ */
+void oracle_linear(const double* x, const double* w, const double* bias, double* out,
+                   int64_t M, int32_t N, int32_t K, int32_t act, const double* res,
+                   const double* alpha, int64_t rows_per_group) {
+  const double c = sqrt(2.0 / 3.14159265358979323846);
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int32_t n = 0; n < N; ++n) {
+      double y = 0.0;
+      for (int32_t k = 0; k < K; ++k) y += x[m * K + k] * w[(int64_t)n * K + k];
+      if (bias) y += bias[n];
+      if (act == 1) y = 0.5 * y * (1.0 + tanh(c * (y + 0.044715 * y * y * y)));
+      if (res) y = res[m * N + n] + alpha[(m / rows_per_group) * N + n] * y;
+      out[m * N + n] = y;
+    }
+  }
+}
+
+/*
  * 3D rotary position embedding (page 2, "3D-RoPE e atencao espaco-temporal").
  * The head dimension is cut into three contiguous bands [t | h | w] of widths
  * d_t, d_h, d_w (each even, summing to d). Within band a, the pair

@@ -187,6 +187,40 @@ def test_euler_zero_step_is_identity_and_steps_compose():
     np.testing.assert_allclose(two, oracle.flow_euler_step(x, u, a + b, 2), atol=1e-14)
 
 
+# ----------------------------------------------------------------------------- linear layers
+# Cost page, "Matematica por tras": Y = X W; DiT page: projections and MLP inside the
+# adaLN-Zero residuals. GELU's tanh form and the bias are this library's reading.
+
+def test_linear_equals_library_matmul_with_bias():
+    rng = np.random.default_rng(11)
+    x, w, b = rng.standard_normal((7, 24)), rng.standard_normal((10, 24)), rng.standard_normal(10)
+    np.testing.assert_allclose(oracle.linear(x, w, b), x @ w.T + b, rtol=1e-13, atol=1e-13)
+
+
+def test_linear_identity_weight_and_gate():
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal((6, 8))
+    np.testing.assert_array_equal(oracle.linear(x, np.eye(8)), x)
+    # adaLN-Zero: a zero gate returns the residual; gate 1 with w = -I cancels it
+    alpha0 = np.zeros((3, 8))
+    np.testing.assert_array_equal(oracle.linear(x, np.eye(8), res=x, alpha=alpha0, rows_per_group=2), x)
+    np.testing.assert_array_equal(oracle.linear(x, -np.eye(8), res=x, alpha=np.ones((3, 8)),
+                                                rows_per_group=2), np.zeros_like(x))
+    # gate group index: group g scales its rows only
+    alpha = np.repeat(np.array([[1.0], [2.0], [3.0]]), 8, axis=1)
+    out = oracle.linear(x, np.eye(8), res=np.zeros_like(x), alpha=alpha, rows_per_group=2)
+    np.testing.assert_array_equal(out, x * np.repeat([1.0, 2.0, 3.0], 2)[:, None])
+
+
+def test_gelu_tanh_form_matches_library_and_its_odd_part():
+    y = np.linspace(-6, 6, 97)
+    got = oracle.linear(y[:, None], np.ones((1, 1)), act=1)[:, 0]
+    ref = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+    # gelu(y) - gelu(-y) = y exactly for the tanh form
+    np.testing.assert_allclose(got - got[::-1], y, atol=1e-12)
+
+
 def test_rope_preserves_norm():
     # Orthogonal rotations (DiT page, 3D-RoPE section): |R q| = |q| per head.
     gh, gw, T, H, d = 3, 5, 4, 3, 64
