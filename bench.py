@@ -198,6 +198,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=24, help="oracle sample rows per step")
     ap.add_argument("--cpu-rows", type=int, default=64, help="oracle rows for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-linear", action="store_true",
+                    help="skip timing the block's linear layers (separate components)")
     ap.add_argument("--rope-mode", default="prepass", choices=["prepass", "fused", "none"],
                     help="prepass: dit_rope3d_qk into scratch, then attention (the product "
                          "path, fastest); fused: RoPE inside the attention kernel (no scratch); "
@@ -322,6 +324,51 @@ def main():
     dit3d.dit_check_device()
     t_euler = statistics.mean(a.elapsed_time(b) for a, b in ee)
 
+    # the block's linear layers (projections with the fused adaLN-Zero gate, MLP up with
+    # GELU), timed on their own: not part of the step; cuBLAS on the same shapes for context
+    lin = {}
+    pk = _peaks()
+    if not args.no_linear:
+        gen = torch.Generator(device="cuda").manual_seed(args.seed + 7)
+        hidden = 4 * D
+        shapes = {"linear_qkv": (3 * D, D, False, False), "linear_out_gated": (D, D, False, True),
+                  "linear_mlp_up_gelu": (hidden, D, True, False)}
+        alpha_g = (torch.randn(rows // rpg, D, device="cuda", generator=gen) * 0.1).to(torch.bfloat16)
+        for name, (n_out, k_in, gelu, gated) in shapes.items():
+            wt = (torch.randn(n_out, k_in, device="cuda", generator=gen) * k_in ** -0.5).to(torch.bfloat16)
+            xin = u if k_in == D else None
+            y = torch.empty(rows, n_out, dtype=torch.bfloat16, device="cuda")
+            kw = dict(gelu=gelu, out=y)
+            if gated:
+                kw.update(residual=dev["x"], alpha=alpha_g, rows_per_group=rpg, out=x_next)
+            run = lambda: dit3d.dit_linear(xin, wt, **kw)
+            for _ in range(2):
+                run()
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(5)]
+            for a, b in pairs:
+                a.record(stream)
+                run()
+                b.record(stream)
+            torch.cuda.synchronize()
+            dit3d.dit_check_device()
+            ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+            fl = 2.0 * rows * n_out * k_in
+            # cuBLAS (torch.matmul) on the same product, no epilogue: context only
+            for _ in range(2):
+                torch.matmul(xin, wt.t())
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for _ in range(5):
+                torch.matmul(xin, wt.t())
+            c1.record(stream)
+            torch.cuda.synchronize()
+            ms_cublas = c0.elapsed_time(c1) / 5
+            lin[name] = {"ms": ms, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "shape": [rows, n_out, k_in],
+                         "frac_burst": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                         "cublas_ms": ms_cublas, "in_step": False}
+            del wt, y
+
     # end to end: pinned host inputs -> device, the path, result -> pinned host
     e2e_keys = ("x", "q", "k", "v", "gamma", "beta", "alpha")
     dev2 = {k: torch.empty_like(dev[k]) for k in e2e_keys}
@@ -349,7 +396,6 @@ def main():
     value = job_throughput(flops, world, ms_step)
     e2e_value = job_throughput(flops, world, e2e_ms)
 
-    pk = _peaks()
     att_tflops = flops / (t_att * 1e-3) / 1e12
     mod_bytes = 4.0 * rows * D
     res_bytes = 6.0 * rows * D
@@ -403,6 +449,7 @@ def main():
                                     "frac_hbm": res_bytes / (t_euler * 1e-3) / 1e9 / pk["hbm_gbs"],
                                     "bytes": res_bytes, "in_step": False,
                                     "note": "sampler update x += dt_frame * u, timed separately"},
+                **lin,
             },
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

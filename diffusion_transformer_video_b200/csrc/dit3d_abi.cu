@@ -19,6 +19,7 @@
 #include "attn_fwd_2sm.cuh"
 #include "common.cuh"
 #include "flow_euler.cuh"
+#include "linear.cuh"
 #include "rope3d.cuh"
 
 using namespace dit3d;
@@ -403,6 +404,53 @@ int dit_flow_euler_step(const void* x, const void* u, const float* dt, void* out
           static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(u), dt,
           static_cast<__nv_bfloat16*>(out), D, rows_per_group);
   }
+  return launch_status();
+}
+
+int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_t M, int32_t N,
+               int32_t K, int32_t activation, const void* residual, const void* alpha,
+               int64_t rows_per_group, void* stream) {
+  if (!x || !w || !out || (residual && !alpha)) return DIT_ERR_NULL;
+  if (M < 0 || M >= (int64_t(1) << 31) || N <= 0 || K <= 0 || (N % 8) || (K % 8) ||
+      (activation != 0 && activation != 1))
+    return DIT_ERR_SHAPE;
+  if (residual && (rows_per_group <= 0 || (M % rows_per_group) != 0)) return DIT_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out) || (bias && !aligned16(bias)) ||
+      (residual && (!aligned16(residual) || !aligned16(alpha))))
+    return DIT_ERR_ALIGN;
+  if (int s = check_device()) return s;
+  if (M == 0) return DIT_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, x, M, K, lin::kBM) || !make_tmap(&tb, w, N, K, lin::kBN)) return DIT_ERR_LAUNCH;
+  lin::Params prm{};
+  prm.bias = static_cast<const __nv_bfloat16*>(bias);
+  prm.res = static_cast<const __nv_bfloat16*>(residual);
+  prm.alpha = static_cast<const __nv_bfloat16*>(alpha);
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.M = M;
+  prm.N = N;
+  prm.K = K;
+  prm.act = activation;
+  prm.rows_per_group = residual ? rows_per_group : 1;
+  prm.tiles_m = static_cast<int32_t>((M + lin::kBM - 1) / lin::kBM);
+  prm.tiles_n = (N + lin::kBN - 1) / lin::kBN;
+  prm.k_blocks = (K + lin::kBK - 1) / lin::kBK;
+  prm.force_timeout = g_force_timeout;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_set[64] = {};
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(lin::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(lin::kSmemBytes)) != cudaSuccess)
+      return DIT_ERR_LAUNCH;
+    attr_set[dev] = true;
+  }
+  const int64_t tiles = static_cast<int64_t>(prm.tiles_m) * prm.tiles_n;
+  if (tiles >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms > 0 ? sms : 148));
+  lin::linear_kernel<<<grid, lin::kThreads, lin::kSmemBytes, st>>>(ta, tb, prm);
   return launch_status();
 }
 

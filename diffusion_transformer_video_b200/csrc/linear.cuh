@@ -1,0 +1,271 @@
+// Linear layers of the DiT block on tcgen05, with fused epilogues.
+//
+//   y = x w^T (+ bias)            "Por que e absurdamente dificil gerar um filme inteiro
+//                                 usando IA", section "Matematica por tras": Y = X W
+//   y = gelu(y)    (optional)     the MLP of "DiT, Flow Matching e 3D Attention",
+//                                 section "A ruptura da U-Net" (tanh form: a reading)
+//   out = res + alpha_g * y       the adaLN-Zero gate of the same section (optional)
+//
+// x [M, K] and w [N, K] bf16 (w in the [out, in] layout of a linear layer), fp32
+// accumulation in tensor memory, bf16 out. The gate fuses the block's residual update
+// into the projection's epilogue, so the attention output projection and the second
+// MLP layer write the block output directly.
+//
+// Persistent kernel, one CTA per SM, 128 x 256 output tiles in grouped order (16
+// M-tiles share each sweep over N, so the A rows and B columns of one wave stay in
+// L2). 256 threads:
+//   warp 0     TMA producer: A (128 x 64) and B (256 x 64) boxes with the 128-byte
+//              swizzle into a 4-stage ring (48 KB per stage)
+//   warp 1     TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma
+//              M128 N256 K16 per stage into one of two 256-column accumulators
+//   warps 4-7  epilogue: thread = output row = TMEM lane; tcgen05.ld 32 columns at a
+//              time, bias / GELU / gate in fp32, one bf16 rounding, 16-byte stores
+// The two accumulators let the epilogue of tile i overlap the main loop of tile i+1.
+// Every mbarrier wait is bounded; on expiry the CTA drains its copies and MMAs, frees
+// its tensor memory and reports DIT_ERR_TIMEOUT through the device error word.
+#pragma once
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace dit3d {
+namespace lin {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kGroupM = 16;
+constexpr uint32_t kABytes = kBM * kBK * 2;            // 16 KB
+constexpr uint32_t kBBytes = kBN * kBK * 2;            // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;    // 48 KB
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024;
+constexpr uint32_t kTmemCols = 2 * kBN;
+
+struct Params {
+  const __nv_bfloat16* bias;   // [N] or null
+  const __nv_bfloat16* res;    // [M, N] or null (then out = y)
+  const __nv_bfloat16* alpha;  // [M / rows_per_group, N] when res is given
+  __nv_bfloat16* out;          // [M, N]
+  int64_t M;
+  int32_t N, K;
+  int32_t act;                 // 0: none, 1: GELU (tanh form)
+  int64_t rows_per_group;
+  int32_t tiles_m, tiles_n, k_blocks;
+  int32_t force_timeout;
+};
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& tm, int& tn) {
+  const int per_group = kGroupM * p.tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * kGroupM;
+  const int gm = min(kGroupM, p.tiles_m - first_m);
+  const int r = t - g * per_group;
+  tm = first_m + r % gm;
+  tn = r / gm;
+}
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float c = 0.7978845608028654f;  // sqrt(2 / pi)
+  const float u = c * fmaf(0.044715f * y, y * y, y);
+  return 0.5f * y * (1.f + tanh_approx(u));
+}
+
+// Epilogue of 8 consecutive columns (one 16-byte store) of one row.
+__device__ __forceinline__ uint4 epilogue8(const float* acc, const Params& p, int64_t row, int col) {
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = acc[e];
+  if (p.bias != nullptr) {
+    const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
+    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      y[2 * e] += bf16lo(bw[e]);
+      y[2 * e + 1] += bf16hi(bw[e]);
+    }
+  }
+  if (p.act == 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = gelu_tanh(y[e]);
+  }
+  uint32_t o[4];
+  if (p.res != nullptr) {
+    const uint4 rv = *reinterpret_cast<const uint4*>(p.res + row * p.N + col);
+    const uint4 av = __ldg(reinterpret_cast<const uint4*>(p.alpha + (row / p.rows_per_group) * p.N + col));
+    const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w}, aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      // a zero gate returns the residual's bits (the adaLN-Zero identity)
+      const float a0 = bf16lo(aw[e]), a1 = bf16hi(aw[e]);
+      const float r0 = bf16lo(rw[e]), r1 = bf16hi(rw[e]);
+      const float o0 = a0 == 0.f ? r0 : fmaf(a0, y[2 * e], r0);
+      const float o1 = a1 == 0.f ? r1 : fmaf(a1, y[2 * e + 1], r1);
+      o[e] = pack_bf16x2(o0, o1);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+              const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tiles = p.tiles_m * p.tiles_n;
+  volatile int* abort = &s_abort;
+
+  if (tid == 0) {
+    s_abort = p.force_timeout ? 1 : 0;
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_u32(&acc_full[b]), 1);
+      ptx::mbar_init(ptx::smem_u32(&acc_empty[b]), kBM);
+    }
+    ptx::mbar_init(ptx::smem_u32(&drain), 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(&s_tmem), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_a);
+      ptx::prefetch_tmap(&tm_b);
+      int it = 0;
+      bool ok = !*abort;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        int tm, tn;
+        tile_coords(t, p, tm, tn);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages;
+          if (it >= kStages &&
+              !ptx::mbar_wait(ptx::smem_u32(&empty[s]), ((it / kStages) - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t f = ptx::smem_u32(&full[s]);
+          const uint32_t dst = ptx::smem_u32(smem + s * kStageBytes);
+          ptx::mbar_arrive_expect_tx(f, kStageBytes);
+          ptx::tma_load_2d(dst, &tm_a, kb * kBK, tm * kBM, f);
+          ptx::tma_load_2d(dst + kABytes, &tm_b, kb * kBK, tn * kBN, f);
+        }
+      }
+      // no copy may still be in flight into shared memory when the CTA exits
+      volatile int never = 0;
+      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
+        ptx::mbar_wait(ptx::smem_u32(&full[j % kStages]), (j / kStages) & 1, &never);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::make_idesc_bf16_f32(kBM, kBN, false);
+      int it = 0, local = 0;
+      bool ok = true, issued = false;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++local) {
+        const int b = local & 1;
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * kBN);
+        if (local >= 2 &&
+            !ptx::mbar_wait(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages;
+          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(smem + s * kStageBytes), b0 = a0 + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::umma_ss(acc, ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B),
+                         ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B), idesc,
+                         (kb > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_commit(ptx::smem_u32(&empty[s]));
+          issued = true;
+        }
+        if (!ok) break;
+        ptx::umma_commit(ptx::smem_u32(&acc_full[b]));
+      }
+      if (issued) {
+        // every MMA of this CTA completes before tensor memory is released
+        volatile int never = 0;
+        ptx::umma_commit(ptx::smem_u32(&drain));
+        ptx::mbar_wait(ptx::smem_u32(&drain), 0, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ================================================================ epilogue
+    const int r = tid - 128;  // row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    int local = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
+      const int b = local & 1;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&acc_full[b]), (local / 2) & 1, abort)))
+        break;
+      ptx::tc_fence_after();
+      int tm, tn;
+      tile_coords(t, p, tm, tn);
+      const int64_t row = static_cast<int64_t>(tm) * kBM + r;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tmem + static_cast<uint32_t>(b * kBN + c * 32) + lane_base, v);
+        ptx::tmem_wait_ld();
+        const int col0 = tn * kBN + c * 32;
+        if (row_ok) {
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            const int col = col0 + g8 * 8;
+            if (col < p.N) {
+              float acc8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc8[e] = __uint_as_float(v[g8 * 8 + e]);
+              *reinterpret_cast<uint4*>(p.out + row * p.N + col) = epilogue8(acc8, p, row, col);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_u32(&acc_empty[b]));
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort) atomicOr(&g_device_error, kDevErrTimeout);
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace lin
+}  // namespace dit3d

@@ -21,8 +21,8 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
                 7: "DIT_ERR_TIMEOUT", 8: "DIT_ERR_ALLOC", 9: "DIT_ERR_SCRATCH"}
 
 # every symbol include/dit3d.h declares
-EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_rope3d_qk",
-           "dit_attn_fwd",
+EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_linear",
+           "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout")
 
@@ -61,6 +61,7 @@ def lib():
         L.dit_adaln_modulate.argtypes = [P, P, P, P, i64, i32, i64, f32, f32, P]
         L.dit_gated_residual.argtypes = [P, P, P, P, i64, i32, i64, P]
         L.dit_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64, P]
+        L.dit_linear.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64, P]
         L.dit_rope3d_qk.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
                                     ctypes.POINTER(RopeDesc), P]
         L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
@@ -168,6 +169,27 @@ def dit_flow_euler_step(x, u, dt, rows_per_group, out=None):
         return out
     _check(lib().dit_flow_euler_step(_ptr(x), _ptr(u), _ptr(dt), _ptr(out), rows, D,
                                      int(rows_per_group), _stream()))
+    return out
+
+
+def dit_linear(x, w, bias=None, gelu=False, residual=None, alpha=None, rows_per_group=1,
+               out=None):
+    """out = [residual + alpha_g *] act(x w^T [+ bias]); x [M, K], w [N, K], bias [N],
+    residual [M, N], alpha [G, N], all bf16 on the device."""
+    _bf16(x, "x")
+    _bf16(w, "w")
+    for t, n in ((bias, "bias"), (residual, "residual"), (alpha, "alpha")):
+        if t is not None:
+            _bf16(t, n)
+    M, K = x.shape
+    N = w.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _bf16(out, "out")
+    if M == 0:
+        return out
+    opt = lambda t: None if t is None else _ptr(t)
+    _check(lib().dit_linear(_ptr(x), _ptr(w), opt(bias), _ptr(out), M, N, K, 1 if gelu else 0,
+                            opt(residual), opt(alpha), int(rows_per_group), _stream()))
     return out
 
 

@@ -7,6 +7,7 @@
  *   o   = softmax(q_rot k_rot^T / sqrt(d_head)) v             dit_attn_fwd
  *   out = x + alpha_g * y                                     dit_gated_residual
  *   x  += dt_frame * u   (sampler step, not in the block)       dit_flow_euler_step
+ *   out = res + alpha_g * act(x w^T + b)  (projections, MLP)     dit_linear
  *
  * Formulas: "DiT, Flow Matching e 3D Attention: A Engenharia de Video com IA",
  * sections "A ruptura da U-Net" (adaLN-Zero) and "3D-RoPE e atencao
@@ -104,6 +105,24 @@ int dit_gated_residual(const void* x, const void* y, const void* alpha, void* ou
  * Errors: as dit_adaln_modulate; DIT_ERR_NULL for a null pointer. */
 int dit_flow_euler_step(const void* x, const void* u, const float* dt, void* out, int64_t rows,
                         int32_t D, int64_t rows_per_group, void* stream);
+
+/* Linear layer of the block with fused epilogue (cost page, "Matematica por tras":
+ * Y = X W; DiT page, "A ruptura da U-Net": the projections and the MLP inside the
+ * adaLN-Zero residuals):
+ *   y   = x w^T + bias                 x [M, K], w [N, K] (linear-layer [out, in] layout)
+ *   y   = gelu(y) if activation == 1   tanh form y/2 (1 + tanh(sqrt(2/pi)(y + 0.044715 y^3)))
+ *   out = residual + alpha[g] * y      if residual != NULL (g = row / rows_per_group;
+ *                                      alpha[g, n] == 0 returns residual's bits), else y
+ * bf16 in and out, fp32 accumulation in tensor memory, one bf16 rounding. bias [N]
+ * may be NULL. residual [M, N] (may alias out), alpha [M / rows_per_group, N].
+ * The GELU and the bias are this library's reading: the pages name only "MLP".
+ * Errors: DIT_ERR_NULL (x, w, out, or alpha with residual); DIT_ERR_SHAPE unless
+ * 0 <= M < 2^31, N > 0, K > 0, N % 8 == 0, K % 8 == 0, activation in {0, 1} and, with
+ * a residual, rows_per_group > 0 dividing M; DIT_ERR_ALIGN for a pointer not 16-byte
+ * aligned. M == 0 is a no-op. */
+int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_t M, int32_t N,
+               int32_t K, int32_t activation, const void* residual, const void* alpha,
+               int64_t rows_per_group, void* stream);
 
 /* Standalone 3D-RoPE of q and k (DiT page, "3D-RoPE e atencao espaco-temporal"),
  * fp32 rotation of bf16 data, the same rotation for every head.

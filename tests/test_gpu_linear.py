@@ -1,0 +1,79 @@
+"""Parity of dit_linear (tcgen05 GEMM with bias / GELU / adaLN-Zero gate epilogues)
+against the fp64 oracle, on single tiles, ragged M/N/K, several waves of the
+persistent grid, and the gate's zero-identity."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from diffusion_transformer_video_b200 import dit3d, workloads as wl
+from tests.helpers import check_modulation, f64, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+RNG = np.random.default_rng(31)
+
+
+def bits(shape, std=1.0):
+    return wl.f32_to_bf16_bits((RNG.standard_normal(shape) * std).astype(np.float32))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 8, 8), (300, 520, 200), (1000, 1024, 512),
+                                   (4096, 768, 1024), (77, 3072, 136)])
+@pytest.mark.parametrize("mode", ["plain", "bias_gelu", "gated"])
+def test_linear_parity(M, N, K, mode):
+    x, w = bits((M, K)), bits((N, K), std=K ** -0.5)
+    kw = {}
+    ref_kw = {}
+    if mode == "bias_gelu":
+        b = bits((N,), std=0.5)
+        kw = dict(bias=to_dev(b), gelu=True)
+        ref_kw = dict(bias=f64(b), act=1)
+    elif mode == "gated":
+        rpg = next(r for r in (64, 7, 1) if M % r == 0)
+        res, alpha = bits((M, N)), bits((M // rpg, N), std=0.5)
+        alpha[0] = 0  # the first group's gate is zero: its rows must be the residual's bits
+        kw = dict(residual=to_dev(res), alpha=to_dev(alpha), rows_per_group=rpg)
+        ref_kw = dict(res=f64(res), alpha=f64(alpha), rows_per_group=rpg)
+    out = dit3d.dit_linear(to_dev(x), to_dev(w), **kw)
+    dit3d.dit_check_device()
+    ref = oracle.linear(f64(x), f64(w), **ref_kw)
+    check_modulation(from_dev(out), ref, f"linear {mode} {M}x{N}x{K}")
+    if mode == "gated":
+        np.testing.assert_array_equal(out[:rpg].view(torch.int16).cpu().numpy(),
+                                      res[:rpg].view(np.int16))
+
+
+def test_linear_in_place_residual_and_errors():
+    M, N, K = 256, 512, 256
+    x, w, res, alpha = bits((M, K)), bits((N, K), std=K ** -0.5), bits((M, N)), bits((2, N))
+    r_dev = to_dev(res)
+    ref = dit3d.dit_linear(to_dev(x), to_dev(w), residual=r_dev, alpha=to_dev(alpha), rows_per_group=128)
+    dit3d.dit_linear(to_dev(x), to_dev(w), residual=r_dev, alpha=to_dev(alpha), rows_per_group=128,
+                     out=r_dev)
+    dit3d.dit_check_device()
+    assert torch.equal(ref, r_dev)
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_linear(to_dev(x), to_dev(bits((12, K))))  # N % 8 != 0
+    assert e.value.status == 2
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_linear(to_dev(x), to_dev(w), residual=r_dev, alpha=to_dev(alpha), rows_per_group=100)
+    assert e.value.status == 2
+    L = dit3d.lib()
+    assert L.dit_linear(None, None, None, None, 1, 8, 8, 0, None, None, 1, None) == 1
+
+
+def test_linear_bounded_wait_reports_timeout():
+    x = torch.randn(512, 256, device="cuda").to(torch.bfloat16)
+    w = torch.randn(512, 256, device="cuda").to(torch.bfloat16)
+    dit3d.lib().dit_debug_force_timeout(1)
+    try:
+        dit3d.dit_linear(x, w)
+        with pytest.raises(dit3d.DitError) as e:
+            dit3d.dit_check_device()
+        assert e.value.status == 7
+    finally:
+        dit3d.lib().dit_debug_force_timeout(0)
+    o = dit3d.dit_linear(x, w)
+    dit3d.dit_check_device()
+    ref = (x.float() @ w.float().T)
+    assert (o.float() - ref).abs().max().item() < 0.5
