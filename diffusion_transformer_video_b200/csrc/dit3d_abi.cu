@@ -28,6 +28,7 @@ namespace {
 
 std::mutex g_mu;
 int g_force_timeout = 0;
+int g_linear_variant = 0;  // 0: one CTA per 128x256 tile; 1: CTA pairs per 256x256 tile
 int g_attn_variant = 0;  // 0: one CTA per query-tile pair; 1: CTA pairs (head_dim 128)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -449,9 +450,32 @@ int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_
   }
   const int64_t tiles = static_cast<int64_t>(prm.tiles_m) * prm.tiles_n;
   if (tiles >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms > 0 ? sms : 148));
+  if (sms <= 0) sms = 148;
+  if (g_linear_variant == 1) {
+    // CTA pairs: 256 x 256 tiles, each CTA loads 128 rows of A and of B
+    CUtensorMap tb2;
+    if (!make_tmap(&tb2, w, N, K, lin::kBM)) return DIT_ERR_LAUNCH;
+    static bool attr2_set[64] = {};
+    if (dev < 64 && !attr2_set[dev]) {
+      if (cudaFuncSetAttribute(lin::linear_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(lin::kSmemBytes2)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+      attr2_set[dev] = true;
+    }
+    const int64_t pair_tiles = static_cast<int64_t>((prm.tiles_m + 1) / 2) * prm.tiles_n;
+    const unsigned grid = 2u * static_cast<unsigned>(std::min<int64_t>(pair_tiles, sms / 2));
+    lin::linear_pair_kernel<<<grid, lin::kThreads, lin::kSmemBytes2, st>>>(ta, tb2, prm);
+    return launch_status();
+  }
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));
   lin::linear_kernel<<<grid, lin::kThreads, lin::kSmemBytes, st>>>(ta, tb, prm);
   return launch_status();
+}
+
+int dit_set_linear_variant(int variant) {
+  if (variant != 0 && variant != 1) return DIT_ERR_SHAPE;
+  g_linear_variant = variant;
+  return DIT_OK;
 }
 
 int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,

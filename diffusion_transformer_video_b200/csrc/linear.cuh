@@ -267,5 +267,222 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
   }
 }
 
+// ---------------------------------------------------------------------------------
+// CTA-pair form (cta_group::2): a cluster of two CTAs computes a 256 x 256 output
+// tile with M = 256 MMAs issued by the even CTA. Each CTA loads its own 128 rows of A
+// and one half (128 rows) of the B tile, so a k-block costs each SM 32 KB of loads
+// instead of 48 KB, and the 6-stage ring holds more k-blocks in flight. Each CTA's
+// TMEM holds its 128 rows x 256 columns (two buffers). Readiness crosses the pair
+// through the even CTA's barriers: a relay thread in each CTA waits for its own
+// stage to land and arrives (release, cluster scope) on the even CTA's ready[s]; the
+// MMA commits arrive on both CTAs' barriers (multicast commit); the epilogue of each
+// CTA signals the even CTA's acc_empty[b] once its 128 threads have drained buffer b.
+// No load is multicast. Measured on B200 at the 480P projection shapes: 2.3x slower
+// than the single-CTA form (601 against 1401 TFLOP/s), so it is not the default.
+constexpr int kStages2 = 6;
+constexpr int kGroupM2 = 8;                            // pair tiles (256 rows) per group
+constexpr uint32_t kHalfBytes = kBM * kBK * 2;         // 16 KB: A half or B half
+constexpr uint32_t kStageBytes2 = 2 * kHalfBytes;      // 32 KB per CTA per stage
+constexpr uint32_t kSmemBytes2 = kStages2 * kStageBytes2 + 1024;
+
+__device__ __forceinline__ void pair_tile_coords(int t, const Params& p, int& tp, int& tn) {
+  const int tiles_p = (p.tiles_m + 1) / 2;
+  const int per_group = kGroupM2 * p.tiles_n;
+  const int g = t / per_group;
+  const int first = g * kGroupM2;
+  const int gm = min(kGroupM2, tiles_p - first);
+  const int r = t - g * per_group;
+  tp = first + r % gm;
+  tn = r / gm;
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                   const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t full[kStages2], ready[kStages2], empty[kStages2], acc_full[2],
+      acc_empty[2], drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+  const int n_tiles = ((p.tiles_m + 1) / 2) * p.tiles_n;
+  volatile int* abort = &s_abort;
+
+  if (tid == 0) {
+    s_abort = p.force_timeout ? 1 : 0;
+    for (int s = 0; s < kStages2; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&ready[s]), 2);
+      ptx::mbar_init(ptx::smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(ptx::smem_u32(&acc_full[b]), 1);
+      ptx::mbar_init(ptx::smem_u32(&acc_empty[b]), 2);
+    }
+    ptx::mbar_init(ptx::smem_u32(&drain), 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) ptx::tmem_alloc_pair(ptx::smem_u32(&s_tmem), kTmemCols);
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync_all();  // both CTAs' barriers and tensor memory exist from here on
+  ptx::tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  // one arrival on the even CTA's copy of barrier `bar`
+  auto arrive_leader = [&](uint64_t* bar) {
+    const uint32_t a = ptx::smem_u32(bar);
+    if (leader) ptx::mbar_arrive(a);
+    else ptx::mbar_arrive_cluster(ptx::mapa_shared(a, 0));
+  };
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_a);
+      ptx::prefetch_tmap(&tm_b);
+      int it = 0;
+      bool ok = !*abort;
+      for (int t = cluster; ok && t < n_tiles; t += n_clusters) {
+        int tp, tn;
+        pair_tile_coords(t, p, tp, tn);
+        const int ya = tp * 2 * kBM + static_cast<int>(rank) * kBM;
+        const int yb = tn * kBN + static_cast<int>(rank) * kBM;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages2;
+          if (it >= kStages2 &&
+              !ptx::mbar_wait_cluster(ptx::smem_u32(&empty[s]), ((it / kStages2) - 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t f = ptx::smem_u32(&full[s]);
+          const uint32_t dst = ptx::smem_u32(smem + s * kStageBytes2);
+          ptx::mbar_arrive_expect_tx(f, kStageBytes2);
+          ptx::tma_load_2d(dst, &tm_a, kb * kBK, ya, f);
+          ptx::tma_load_2d(dst + kHalfBytes, &tm_b, kb * kBK, yb, f);
+        }
+      }
+      volatile int never = 0;
+      for (int j = (it > kStages2 ? it - kStages2 : 0); j < it; ++j)
+        ptx::mbar_wait(ptx::smem_u32(&full[j % kStages2]), (j / kStages2) & 1, &never);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ================================================================ relay
+    // this CTA's stage landed -> one arrival on the even CTA's ready[s]
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int t = cluster; ok && t < n_tiles; t += n_clusters)
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages2;
+          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages2) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          arrive_leader(&ready[s]);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = ptx::make_idesc_bf16_f32(2 * kBM, kBN, false);
+      int it = 0, local = 0;
+      bool ok = true, issued = false;
+      for (int t = cluster; ok && t < n_tiles; t += n_clusters, ++local) {
+        const int b = local & 1;
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * kBN);
+        if (local >= 2 &&
+            !ptx::mbar_wait_cluster(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % kStages2;
+          if (!ptx::mbar_wait_cluster(ptx::smem_u32(&ready[s]), (it / kStages2) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(smem + s * kStageBytes2), b0 = a0 + kHalfBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::umma_ss_pair(acc, ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B),
+                              ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B), idesc,
+                              (kb > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_commit_pair(ptx::smem_u32(&empty[s]));
+          issued = true;
+        }
+        if (!ok) break;
+        ptx::umma_commit_pair(ptx::smem_u32(&acc_full[b]));
+      }
+      if (issued) {
+        volatile int never = 0;
+        ptx::umma_commit_pair(ptx::smem_u32(&drain));
+        ptx::mbar_wait_cluster(ptx::smem_u32(&drain), 0, &never);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ================================================================ epilogue
+    const int r = tid - 128;
+    const uint32_t lane_base = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    int local = 0;
+    for (int t = cluster; t < n_tiles; t += n_clusters, ++local) {
+      const int b = local & 1;
+      if (!__all_sync(0xffffffffu,
+                      ptx::mbar_wait_cluster(ptx::smem_u32(&acc_full[b]), (local / 2) & 1, abort)))
+        break;
+      ptx::tc_fence_after();
+      int tp, tn;
+      pair_tile_coords(t, p, tp, tn);
+      const int64_t row = static_cast<int64_t>(tp) * 2 * kBM + rank * kBM + r;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tmem + static_cast<uint32_t>(b * kBN + c * 32) + lane_base, v);
+        ptx::tmem_wait_ld();
+        const int col0 = tn * kBN + c * 32;
+        if (row_ok) {
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            const int col = col0 + g8 * 8;
+            if (col < p.N) {
+              float acc8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc8[e] = __uint_as_float(v[g8 * 8 + e]);
+              *reinterpret_cast<uint4*>(p.out + row * p.N + col) = epilogue8(acc8, p, row, col);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      named_sync(1, 128);
+      if (r == 0) arrive_leader(&acc_empty[b]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
+  if (tid == 0 && *abort) atomicOr(&g_device_error, kDevErrTimeout);
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 }  // namespace lin
 }  // namespace dit3d

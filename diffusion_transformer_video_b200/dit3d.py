@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
 
 # every symbol include/dit3d.h declares
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_linear",
+           "dit_set_linear_variant",
            "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout")
@@ -233,6 +234,11 @@ def dit_attn_fwd(q, k, v, n_seq=1, cu_seqlens=None, rope: RopeDesc | None = None
 def dit_set_attn_variant(variant: int):
     """0: single-CTA attention kernel (default); 1: CTA-pair kernel (head_dim 128)."""
     _check(lib().dit_set_attn_variant(int(variant)))
+
+
+def dit_set_linear_variant(variant: int):
+    """0: one CTA per 128x256 tile (default); 1: CTA-pair GEMM on 256x256 tiles."""
+    _check(lib().dit_set_linear_variant(int(variant)))
 
 
 def dit_check_device():

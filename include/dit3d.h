@@ -124,6 +124,14 @@ int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_
                int32_t K, int32_t activation, const void* residual, const void* alpha,
                int64_t rows_per_group, void* stream);
 
+/* Kernel form of dit_linear for later calls in this process: 0 (default) runs one
+ * CTA per 128 x 256 tile, 1 CTA pairs (cta_group::2) on 256 x 256 tiles (correct, but
+ * measured 2.3x slower on B200: every k-block crosses the pair through the even CTA's
+ * barriers). Same results up to the order of fp32 additions. No counterpart in the
+ * source pages.
+ * Errors: DIT_ERR_SHAPE for any other value. */
+int dit_set_linear_variant(int variant);
+
 /* Standalone 3D-RoPE of q and k (DiT page, "3D-RoPE e atencao espaco-temporal"),
  * fp32 rotation of bf16 data, the same rotation for every head.
  *   q_in, k_in   : [rows, H, d] bf16; k_in may be NULL (then k_out is ignored)

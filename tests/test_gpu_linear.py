@@ -17,10 +17,17 @@ def bits(shape, std=1.0):
     return wl.f32_to_bf16_bits((RNG.standard_normal(shape) * std).astype(np.float32))
 
 
+@pytest.fixture(params=[0, 1], ids=["single_cta", "cta_pair"])
+def variant(request):
+    dit3d.dit_set_linear_variant(request.param)
+    yield request.param
+    dit3d.dit_set_linear_variant(0)
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 8, 8), (300, 520, 200), (1000, 1024, 512),
                                    (4096, 768, 1024), (77, 3072, 136)])
 @pytest.mark.parametrize("mode", ["plain", "bias_gelu", "gated"])
-def test_linear_parity(M, N, K, mode):
+def test_linear_parity(variant, M, N, K, mode):
     x, w = bits((M, K)), bits((N, K), std=K ** -0.5)
     kw = {}
     ref_kw = {}
@@ -43,7 +50,7 @@ def test_linear_parity(M, N, K, mode):
                                       res[:rpg].view(np.int16))
 
 
-def test_linear_in_place_residual_and_errors():
+def test_linear_in_place_residual_and_errors(variant):
     M, N, K = 256, 512, 256
     x, w, res, alpha = bits((M, K)), bits((N, K), std=K ** -0.5), bits((M, N)), bits((2, N))
     r_dev = to_dev(res)
@@ -62,7 +69,23 @@ def test_linear_in_place_residual_and_errors():
     assert L.dit_linear(None, None, None, None, 1, 8, 8, 0, None, None, 1, None) == 1
 
 
-def test_linear_bounded_wait_reports_timeout():
+def test_linear_variants_agree():
+    M, N, K = 700, 1280, 960
+    x, w = to_dev(bits((M, K))), to_dev(bits((N, K), std=K ** -0.5))
+    outs = []
+    for v in (0, 1):
+        dit3d.dit_set_linear_variant(v)
+        outs.append(dit3d.dit_linear(x, w))
+    dit3d.dit_set_linear_variant(0)
+    dit3d.dit_check_device()
+    # same products, fp32 sums in possibly different order: within one bf16 ulp
+    diff = (outs[0].float() - outs[1].float()).abs()
+    assert (diff <= outs[0].float().abs() * 2 ** -7 + 1e-6).all()
+    with pytest.raises(dit3d.DitError):
+        dit3d.dit_set_linear_variant(3)
+
+
+def test_linear_bounded_wait_reports_timeout(variant):
     x = torch.randn(512, 256, device="cuda").to(torch.bfloat16)
     w = torch.randn(512, 256, device="cuda").to(torch.bfloat16)
     dit3d.lib().dit_debug_force_timeout(1)
