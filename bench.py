@@ -332,11 +332,13 @@ def main():
         gen = torch.Generator(device="cuda").manual_seed(args.seed + 7)
         hidden = 4 * D
         shapes = {"linear_qkv": (3 * D, D, False, False), "linear_out_gated": (D, D, False, True),
-                  "linear_mlp_up_gelu": (hidden, D, True, False)}
+                  "linear_mlp_up_gelu": (hidden, D, True, False),
+                  "linear_mlp_down_gated": (D, hidden, False, True)}
+        h_act = None
         alpha_g = (torch.randn(rows // rpg, D, device="cuda", generator=gen) * 0.1).to(torch.bfloat16)
         for name, (n_out, k_in, gelu, gated) in shapes.items():
             wt = (torch.randn(n_out, k_in, device="cuda", generator=gen) * k_in ** -0.5).to(torch.bfloat16)
-            xin = u if k_in == D else None
+            xin = u if k_in == D else h_act
             y = torch.empty(rows, n_out, dtype=torch.bfloat16, device="cuda")
             kw = dict(gelu=gelu, out=y)
             if gated:
@@ -367,6 +369,8 @@ def main():
             lin[name] = {"ms": ms, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "shape": [rows, n_out, k_in],
                          "frac_burst": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
                          "cublas_ms": ms_cublas, "in_step": False}
+            if name == "linear_mlp_up_gelu":
+                h_act = y  # the MLP's hidden activations feed the down projection
             del wt, y
 
     # end to end: pinned host inputs -> device, the path, result -> pinned host
