@@ -70,3 +70,53 @@ def test_workload_attention_sampled(case):
     check_attention(got, ref_o, f"{w.name} attention")
     got_lse = lse[torch.from_numpy(rows).cuda()].cpu().double().numpy()
     np.testing.assert_allclose(got_lse, ref_lse, atol=2e-2)
+
+
+def test_workload_attention_product_step_equals_fused(case):
+    # the benchmark's step rotates q and k in one pass and attends over the rotated
+    # operands; the rotation is the same fp32 arithmetic, so the output has the same bits
+    w, inp = case
+    desc = dit3d.rope_desc(w.grid_h, w.grid_w, w.bands, w.base)
+    cu = w.cu_seqlens if w.varlen else None
+    q, k, v = to_dev(inp["q"]), to_dev(inp["k"]), to_dev(inp["v"])
+    o_fused = dit3d.dit_attn_fwd(q, k, v, n_seq=w.n_seq, cu_seqlens=cu, rope=desc)
+    qr, kr = dit3d.dit_rope3d_qk(q, k, desc, n_seq=w.n_seq, cu_seqlens=cu)
+    o_step = dit3d.dit_attn_fwd(qr, kr, v, n_seq=w.n_seq, cu_seqlens=cu)
+    dit3d.dit_check_device()
+    assert torch.equal(o_fused, o_step)
+
+
+def test_workload_linear_sampled_and_euler(case):
+    w, inp = case
+    D, rows, rpg = w.d_model, w.rows, w.rows_per_group
+    rng = np.random.default_rng(41)
+    x = to_dev(inp["x"])
+    sample = np.unique(np.concatenate([[0, rows - 1], np.arange(max(rows - 130, 0), rows, 7),
+                                       rng.integers(0, rows, 24)]))
+    # QKV-shaped projection with bias
+    wq = wl.f32_to_bf16_bits((rng.standard_normal((3 * D, D)) * D ** -0.5).astype(np.float32))
+    bq = wl.f32_to_bf16_bits((rng.standard_normal(3 * D) * 0.1).astype(np.float32))
+    y = dit3d.dit_linear(x, to_dev(wq), bias=to_dev(bq))
+    dit3d.dit_check_device()
+    got = from_dev(y[torch.from_numpy(sample).cuda()])
+    del y
+    ref = oracle.linear(f64(inp["x"][sample]), f64(wq), bias=f64(bq))
+    check_modulation(got, ref, f"{w.name} qkv projection")
+    # output projection with the gate fused, written over the residual
+    wo = wl.f32_to_bf16_bits((rng.standard_normal((D, D)) * D ** -0.5).astype(np.float32))
+    alpha = wl.make_inputs(w, seed=0, which=("alpha",))["alpha"]
+    h = to_dev(inp["y"])
+    res = x.clone()
+    dit3d.dit_linear(h, to_dev(wo), residual=res, alpha=to_dev(alpha), rows_per_group=rpg, out=res)
+    dit3d.dit_check_device()
+    got = from_dev(res[torch.from_numpy(sample).cuda()])
+    ref = oracle.linear(f64(inp["y"][sample]), f64(wo), res=f64(inp["x"][sample]),
+                        alpha=f64(alpha[sample // rpg]), rows_per_group=1)
+    check_modulation(got, ref, f"{w.name} gated output projection")
+    # one Euler step per frame on the whole latent
+    frame = w.grid_h * w.grid_w
+    dt = rng.uniform(0.0, 0.1, rows // frame).astype(np.float32)
+    xn = dit3d.dit_flow_euler_step(x, h, torch.from_numpy(dt).cuda(), frame)
+    dit3d.dit_check_device()
+    ref = oracle.flow_euler_step(f64(inp["x"]), f64(inp["y"]), dt.astype(np.float64), frame)
+    check_modulation(from_dev(xn), ref, f"{w.name} euler step")
