@@ -35,8 +35,7 @@ sys.path.insert(0, ROOT)
 METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
 UNIT = "TFLOP/s"
 # DRAM bytes per head of one attention launch at the 480P geometry, from an ncu capture
-# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum over 16;
-# profiles/attn_fwd_480p_h16.md), keyed by RoPE mode
+# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum over 16), keyed by RoPE mode
 # ("prepass" and "none" run the same kernel, without in-kernel RoPE). Heads are
 # independent, so a launch's traffic is this times its head count. None where the
 # current kernel has not been captured; other workloads report null.
@@ -138,11 +137,33 @@ def cpu_oracle_attention(w, qkv64, n_rows: int, seed: int = 0):
     return flops / dt / 1e12, dt, sample, threads
 
 
+def resolve_workload(args):
+    """The workload of this run (with --heads applied)."""
+    from diffusion_transformer_video_b200 import workloads as wl
+    w = wl.get_workload(args.workload, args.seed)
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}-h{args.heads}", heads=args.heads)
+    return w
+
+
+def workload_config(w, world: int) -> dict:
+    """The `config` object of the JSON line, the same for both arms."""
+    rows, D = w.rows, w.d_model
+    return {"workload": w.name, "batch": w.n_seq, "seq_len": w.max_seqlen,
+            "rows": rows, "heads": w.heads, "head_dim": w.head_dim, "d_model": D,
+            "rope_bands": list(w.bands), "grid": [w.grid_h, w.grid_w],
+            "parallelism": f"dp{world} (independent batches)",
+            "l2": "inputs larger than L2 (x, q, k, v are %.0f MB each)" % (rows * D * 2 / 1e6)
+            if rows * D * 2 > 126e6 else "inputs smaller than L2 (no flush)",
+            "note": w.note}
+
+
 def run_reference(args, rank, world):
     from diffusion_transformer_video_b200 import workloads as wl
     if rank != 0:
         return
-    w = wl.get_workload(args.workload, args.seed)
+    w = resolve_workload(args)
     inp = wl.make_inputs(w, args.seed, which=("q", "k", "v"))
     qkv64 = widen_qkv(inp)
     n_rows = args.ref_rows
@@ -157,8 +178,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded bf16 N(0,1) inputs widened to fp64)",
-            "config": {"workload": w.name, "rows": w.rows, "heads": w.heads,
-                       "head_dim": w.head_dim, "note": w.note},
+            "config": workload_config(w, world),
             "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": threads,
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -234,10 +254,7 @@ def main():
             dist.barrier()
 
     dit3d.dit_set_attn_variant(args.attn_variant)
-    w = wl.get_workload(args.workload, args.seed)
-    if args.heads:
-        import dataclasses
-        w = dataclasses.replace(w, name=f"{w.name}-h{args.heads}", heads=args.heads)
+    w = resolve_workload(args)
     # every rank runs its own batch of the workload (seeded per rank)
     seed = rank_seed(args.seed, rank)
     inp = wl.make_inputs(w, seed)
@@ -456,13 +473,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded bf16 N(0,1) x/q/k/v, N(0,0.1) adaLN params)",
-            "config": {"workload": w.name, "batch": w.n_seq, "seq_len": w.max_seqlen,
-                       "rows": rows, "heads": H, "head_dim": d, "d_model": D,
-                       "rope_bands": list(w.bands), "grid": [w.grid_h, w.grid_w],
-                       "parallelism": f"dp{world} (independent batches)",
-                       "l2": "inputs larger than L2 (x, q, k, v are %.0f MB each)" % (rows * D * 2 / 1e6)
-                       if rows * D * 2 > 126e6 else "inputs smaller than L2 (no flush)",
-                       "note": w.note},
+            "config": workload_config(w, world),
             "gpu_launches": (4 if args.rope_mode == "prepass" else 3) * K,
             "roofline": {"bound": "tensor", "achieved": att_tflops,
                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",

@@ -7,7 +7,7 @@ import torch
 
 from diffusion_transformer_video_b200 import workloads as wl
 
-# the benchmark spec tolerances: attention max abs 2e-2 / mean abs 2e-3 on unit-normal inputs;
+# Tolerances of the stated accuracy targets: attention max abs 2e-2 / mean abs 2e-3 on unit-normal inputs;
 # modulation kernels 1e-2 max abs, measured as |gpu - ref| <= 1e-2 + half a bf16 ulp of ref
 # (a correctly rounded bf16 output of |ref| >= 4 is already 1/64 away from ref).
 ATTN_MAX, ATTN_MEAN = 2e-2, 2e-3
