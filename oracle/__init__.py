@@ -13,6 +13,8 @@ Each wrapper cites the passage it restates:
   (Euler sampler on the straight path), with the per-frame local times of
   "Flowception: Temporally Expansive Flow Matching for Video Generation",
   section "Metodologia".
+* ``quantize_e4m3`` / ``attn_fwd_qk8`` -- DiT page, section "Engenharia de inferencia e
+  paralelismo de contexto: Ulysses, Ring Attention e FP8" (FP8 E4M3 activations).
 * ``linear`` -- "Por que e absurdamente dificil gerar um filme inteiro usando IA",
   section "Matematica por tras" (Y = X W), with the DiT page's MLP and gates.
 * ``rope3d`` -- same page, section "3D-RoPE e atencao espaco-temporal".
@@ -57,11 +59,14 @@ def _load():
         lib.oracle_gated_residual.argtypes = [P, P, P, P, i64, i32, i64]
         lib.oracle_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64]
         lib.oracle_linear.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64]
+        lib.oracle_quantize_e4m3.argtypes = [P, P, i64, f64]
+        lib.oracle_round_bf16.argtypes = [P, P, i64]
         lib.oracle_rope3d.argtypes = [P, P, i64, i32, i32, P, i32, i32, i32, i32, i32, i32, f64,
                                       i32, i32, i32]
         lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, P, i32, f64, P, i64]
         for f in (lib.oracle_adaln_modulate, lib.oracle_gated_residual, lib.oracle_rope3d,
-                  lib.oracle_attn_fwd, lib.oracle_flow_euler_step, lib.oracle_linear):
+                  lib.oracle_attn_fwd, lib.oracle_flow_euler_step, lib.oracle_linear,
+                  lib.oracle_quantize_e4m3, lib.oracle_round_bf16):
             f.restype = None
         _lib = lib
     return _lib
@@ -139,6 +144,40 @@ def linear(x, w, bias=None, act: int = 0, res=None, alpha=None,
                           int(act), None if r is None else _ptr(r), None if a is None else _ptr(a),
                           rows_per_group)
     return out
+
+
+def quantize_e4m3(x, inv_scale: float = 1.0) -> np.ndarray:
+    """e4m3(x * inv_scale) (nearest, ties to even, saturated at 448) as fp64 values."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    _load().oracle_quantize_e4m3(_ptr(x), _ptr(out), x.size, float(inv_scale))
+    return out
+
+
+def round_bf16(x) -> np.ndarray:
+    """Nearest bf16 value of each element (ties to even), fp64."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    _load().oracle_round_bf16(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def attn_fwd_qk8(q, k, v, cu_seqlens, q_scale: float, k_scale: float, scale: float | None = None,
+                 qrows=None, rope=None):
+    """Attention whose Q K^T runs on FP8 E4M3 operands: q and k (rotated by ``rope3d``
+    and rounded to bf16 first, when ``rope`` is given) are quantised as
+    e4m3(q / q_scale), e4m3(k / k_scale) and the scores use q_scale * k_scale times
+    their product; P and V stay exact. Returns (o, lse) like ``attn_fwd``."""
+    q, k = _f64(q), _f64(k)
+    if rope is not None:
+        cu = _cu(cu_seqlens)
+        q = round_bf16(rope3d(q, cu, rope["grid_h"], rope["grid_w"], rope["bands"],
+                              rope.get("base", 10000.0), rope.get("offsets", (0, 0, 0))))
+        k = round_bf16(rope3d(k, cu, rope["grid_h"], rope["grid_w"], rope["bands"],
+                              rope.get("base", 10000.0), rope.get("offsets", (0, 0, 0))))
+    q8 = quantize_e4m3(q, 1.0 / q_scale) * q_scale
+    k8 = quantize_e4m3(k, 1.0 / k_scale) * k_scale
+    return attn_fwd(q8, k8, v, cu_seqlens, scale=scale, qrows=qrows)
 
 
 def rope3d(v, cu_seqlens, grid_h: int, grid_w: int, bands, base: float = 10000.0,

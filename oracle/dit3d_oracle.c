@@ -133,6 +133,50 @@ void oracle_linear(const double* x, const double* w, const double* bias, double*
 }
 
 /*
+ * FP8 E4M3 quantisation (page 2, "Engenharia de inferencia e paralelismo de contexto:
+ * Ulysses, Ring Attention e FP8": activations quantised to FP8 E4M3/E5M2). E4M3 as
+ * the OCP format defines it: 1 sign, 4 exponent (bias 7) and 3 mantissa bits, no
+ * infinities, normal numbers 2^-6 .. 448 = 1.75 * 2^8, subnormals k * 2^-9. Values are
+ * rounded to nearest, ties to even, and saturated at +-448 (the reading taken for
+ * values beyond the range: clamp, as a per-tensor scale is meant to avoid them).
+ * out[i] = e4m3(x[i] * inv_scale), returned as its real value.
+ */
+static double e4m3_round(double x) {
+  if (x != x) return x;
+  const double a = fabs(x);
+  double q;
+  if (a >= 448.0) {
+    q = 448.0;
+  } else if (a < 0.015625) {  /* below 2^-6: subnormal spacing 2^-9 */
+    q = nearbyint(a * 512.0) / 512.0;
+  } else {
+    int e;
+    frexp(a, &e);                     /* a = f * 2^e, f in [0.5, 1): 2^(e-1) <= a < 2^e */
+    const double quantum = ldexp(1.0, e - 1 - 3);
+    q = nearbyint(a / quantum) * quantum;
+    if (q > 448.0) q = 448.0;
+  }
+  return x < 0 ? -q : q;
+}
+
+void oracle_quantize_e4m3(const double* x, double* out, int64_t n, double inv_scale) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_round(x[i] * inv_scale);
+}
+
+/* Round to the nearest bf16 value (8 significant bits, ties to even). */
+void oracle_round_bf16(const double* x, double* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double a = fabs(x[i]);
+    if (a == 0.0 || x[i] != x[i]) { out[i] = x[i]; continue; }
+    int e;
+    frexp(a, &e);
+    const double quantum = ldexp(1.0, e - 8);
+    const double q = nearbyint(a / quantum) * quantum;
+    out[i] = x[i] < 0 ? -q : q;
+  }
+}
+
+/*
  * 3D rotary position embedding (page 2, "3D-RoPE e atencao espaco-temporal").
  * The head dimension is cut into three contiguous bands [t | h | w] of widths
  * d_t, d_h, d_w (each even, summing to d). Within band a, the pair

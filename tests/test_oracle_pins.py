@@ -221,6 +221,52 @@ def test_gelu_tanh_form_matches_library_and_its_odd_part():
     np.testing.assert_allclose(got - got[::-1], y, atol=1e-12)
 
 
+# ----------------------------------------------------------------------------- FP8 (E4M3)
+# DiT page, "Engenharia de inferencia e paralelismo de contexto: ... FP8": activations in
+# FP8 E4M3. The format (OCP E4M3: bias 7, 3 mantissa bits, max 448) is pinned against
+# torch's float8_e4m3fn conversion inside its range, and saturation by closed form.
+
+def test_e4m3_matches_library_conversion_in_range():
+    rng = np.random.default_rng(13)
+    codes = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    grid = np.sort(codes[np.isfinite(codes)])
+    mids = (grid[1:] + grid[:-1]) / 2                   # exact ties: nearest-even decides
+    x = np.concatenate([grid, mids, rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 0.01])
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(oracle.quantize_e4m3(x), ref)
+
+
+def test_e4m3_saturates_and_scales():
+    np.testing.assert_array_equal(oracle.quantize_e4m3(np.array([449.0, 1e9, -500.0])),
+                                  [448.0, 448.0, -448.0])
+    # inv_scale multiplies before rounding: 3 * 0.5 = 1.5 is exact; 1.2 * 64 = 76.8 lies
+    # in [64, 128), where e4m3 values are 8 apart: 80
+    np.testing.assert_array_equal(oracle.quantize_e4m3(np.array([3.0, 1.2]), 0.5), [1.5, 0.625])
+    np.testing.assert_array_equal(oracle.quantize_e4m3(np.array([1.2]), 64.0), [80.0])
+
+
+def test_bf16_rounding_matches_library():
+    rng = np.random.default_rng(14)
+    x = np.concatenate([rng.standard_normal(5000) * 10.0 ** rng.integers(-6, 6, 5000),
+                        [1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8)]])
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(x), ref)
+
+
+def test_attn_qk8_is_attention_of_the_quantised_operands():
+    rng = np.random.default_rng(15)
+    N, H, d = 40, 2, 32
+    # operands already on the e4m3 grid times a power of two: quantisation is exact
+    q = oracle.quantize_e4m3(rng.standard_normal((N, H, d)) * 8) / 8
+    k = oracle.quantize_e4m3(rng.standard_normal((N, H, d)) * 8) / 8
+    v = rng.standard_normal((N, H, d))
+    cu = np.array([0, N], np.int32)
+    o8, l8 = oracle.attn_fwd_qk8(q, k, v, cu, 1 / 8, 1 / 8)
+    o, l = oracle.attn_fwd(q, k, v, cu)
+    np.testing.assert_allclose(o8, o, atol=1e-13)
+    np.testing.assert_allclose(l8, l, atol=1e-13)
+
+
 def test_rope_preserves_norm():
     # Orthogonal rotations (DiT page, 3D-RoPE section): |R q| = |q| per head.
     gh, gw, T, H, d = 3, 5, 4, 3, 64
