@@ -342,6 +342,39 @@ def main():
     dit3d.dit_check_device()
     t_euler = statistics.mean(a.elapsed_time(b) for a, b in ee)
 
+    # FP8 (E4M3) Q K^T: quantise the rotated q and k (power-of-two scale 1/64, exact
+    # products), then attention with the E4M3 product; timed on its own, not in the step
+    fp8 = None
+    if d == 128 and args.rope_mode == "prepass":
+        q8 = torch.empty(rows, H, d, dtype=torch.uint8, device="cuda")
+        k8 = torch.empty_like(q8)
+        o8 = torch.empty_like(o)
+
+        def fp8_attention():
+            dit3d.dit_quantize_e4m3(q_rot, 64.0, out=q8)
+            dit3d.dit_quantize_e4m3(k_rot, 64.0, out=k8)
+            dit3d.dit_attn_fwd_qk8(q8, k8, dev["v"], 1 / 64, 1 / 64, n_seq=w.n_seq,
+                                   cu_seqlens=cu, out=o8)
+        for _ in range(2):
+            fp8_attention()
+        ev3 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(max(K, 3))]
+        for e in ev3:
+            e[0].record(stream)
+            dit3d.dit_quantize_e4m3(q_rot, 64.0, out=q8)
+            dit3d.dit_quantize_e4m3(k_rot, 64.0, out=k8)
+            e[1].record(stream)
+            dit3d.dit_attn_fwd_qk8(q8, k8, dev["v"], 1 / 64, 1 / 64, n_seq=w.n_seq,
+                                   cu_seqlens=cu, out=o8)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        dit3d.dit_check_device()
+        t_q8 = statistics.mean(e[0].elapsed_time(e[1]) for e in ev3)
+        t_a8 = statistics.mean(e[1].elapsed_time(e[2]) for e in ev3)
+        fp8 = {"ms": t_a8, "TFLOP/s": w.attn_flops() / (t_a8 * 1e-3) / 1e12,
+               "quantize_ms": t_q8, "max_abs_vs_bf16_attention": float((o8.float() - o.float()).abs().max()),
+               "in_step": False, "note": "E4M3 q, k (scale 1/64), bf16 P and V"}
+        del q8, k8, o8
+
     # the block's linear layers (projections with the fused adaLN-Zero gate, MLP up with
     # GELU), timed on their own: not part of the step; cuBLAS on the same shapes for context
     lin = {}
@@ -498,6 +531,7 @@ def main():
                                     "frac_hbm": res_bytes / (t_euler * 1e-3) / 1e9 / pk["hbm_gbs"],
                                     "bytes": res_bytes, "in_step": False,
                                     "note": "sampler update x += dt_frame * u, timed separately"},
+                "attn_fwd_qk8": fp8,
                 **lin,
             },
             "clocks": clocks,

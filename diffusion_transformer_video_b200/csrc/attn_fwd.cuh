@@ -213,11 +213,18 @@ __device__ __forceinline__ void rope_tile_global(uint8_t* tile, int64_t row0, in
   }
 }
 
-template <int D>
+// QK8: q and k arrive as FP8 E4M3 codes (one byte per element, d = 128: one 128-byte
+// swizzle row per token) and S = Q K^T runs as kind::f8f6f4 MMAs (K = 32 each); the
+// host folds the two dequantisation scales into the softmax scale. P and V stay bf16.
+// The tiles keep the bf16 layout's shared-memory slots (half of each is used).
+template <int D, bool QK8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using L = Smem<D>;
+  static_assert(!QK8 || D == 128, "E4M3 Q/K tiles use 128-byte rows (head_dim 128)");
+  constexpr int kQKBoxes = QK8 ? 1 : D / 64;                       // TMA boxes per Q/K tile
+  constexpr uint32_t kQKBytes = QK8 ? kTileM * D : L::kTile;       // bytes per Q/K tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -432,9 +439,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!*abort) {
         if (is_k) {
           ptx::prefetch_tmap(&tm_q);
-          ptx::mbar_arrive_expect_tx(q_full, 2 * L::kTile);
+          ptx::mbar_arrive_expect_tx(q_full, 2 * kQKBytes);
           for (int qi = 0; qi < 2; ++qi)
-            for (int blk = 0; blk < D / 64; ++blk)
+            for (int blk = 0; blk < kQKBoxes; ++blk)
               ptx::tma_load_2d(ptx::smem_u32(smem + (qi ? L::kQ1 : L::kQ0) + blk * 16384), &tm_q,
                                x0 + blk * 64, static_cast<int>(seq_start + q_row0 + qi * kTileM),
                                q_full);
@@ -446,8 +453,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             break;
           const int y = static_cast<int>(seq_start + static_cast<int64_t>(j) * kTileN);
           const uint32_t f = ptx::smem_u32(&full[st]);
-          ptx::mbar_arrive_expect_tx(f, L::kTile);
-          for (int blk = 0; blk < D / 64; ++blk)
+          ptx::mbar_arrive_expect_tx(f, is_k ? kQKBytes : L::kTile);
+          const int boxes = is_k ? kQKBoxes : D / 64;
+          for (int blk = 0; blk < boxes; ++blk)
             ptx::tma_load_2d(ptx::smem_u32(smem + ring + st * L::kTile + blk * 16384), tm,
                              x0 + blk * 64, y, f);
           ++issued;
@@ -471,12 +479,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       auto qk = [&](int qi, int st) {
         const uint32_t qa = sbase + (qi ? L::kQ1 : L::kQ0);
         const uint32_t ka = sbase + L::kK + st * L::kTile;
+        if constexpr (QK8) {
+          constexpr uint32_t idesc_qk8 = ptx::make_idesc_e4m3_f32(kTileM, kTileN);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::umma_ss(tmem + col_s(qi), ptx::make_smem_desc(qa + off, 16, 1024, ptx::kSwizzle128B),
-                       ptx::make_smem_desc(ka + off, 16, 1024, ptx::kSwizzle128B), idesc_qk,
-                       kk > 0);
+          for (int kk = 0; kk < D / 32; ++kk)  // 32 bytes = 32 E4M3 elements per MMA
+            ptx::umma_ss_f8(tmem + col_s(qi),
+                            ptx::make_smem_desc(qa + kk * 32, 16, 1024, ptx::kSwizzle128B),
+                            ptx::make_smem_desc(ka + kk * 32, 16, 1024, ptx::kSwizzle128B),
+                            idesc_qk8, kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            ptx::umma_ss(tmem + col_s(qi), ptx::make_smem_desc(qa + off, 16, 1024, ptx::kSwizzle128B),
+                         ptx::make_smem_desc(ka + off, 16, 1024, ptx::kSwizzle128B), idesc_qk,
+                         kk > 0);
+          }
         }
         ptx::umma_commit(ptx::smem_u32(&b->s_full[qi]));
       };

@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "flow_euler.cuh"
 #include "linear.cuh"
+#include "quant.cuh"
 #include "rope3d.cuh"
 
 using namespace dit3d;
@@ -221,26 +222,41 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+// [rows, cols] bytes (E4M3 codes), boxes of 128 columns x box_rows rows, 128-byte swizzle.
+bool make_tmap8(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
+                uint32_t box_rows = 128) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool QK8 = false>
 int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32_t H,
                 const attn::Params& prm, int n_work, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, rows, static_cast<int64_t>(H) * D) ||
-      !make_tmap(&tk, k, rows, static_cast<int64_t>(H) * D) ||
-      !make_tmap(&tv, v, rows, static_cast<int64_t>(H) * D))
-    return DIT_ERR_LAUNCH;
+  const int64_t cols = static_cast<int64_t>(H) * D;
+  const bool ok_qk = QK8 ? (make_tmap8(&tq, q, rows, cols) && make_tmap8(&tk, k, rows, cols))
+                         : (make_tmap(&tq, q, rows, cols) && make_tmap(&tk, k, rows, cols));
+  if (!ok_qk || !make_tmap(&tv, v, rows, cols)) return DIT_ERR_LAUNCH;
   constexpr uint32_t smem = attn::Smem<D>::kRequest;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(attn::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn::attn_fwd_kernel<D, QK8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return DIT_ERR_LAUNCH;
     attr_set[dev] = true;
   }
   dim3 grid(n_work, H);
-  attn::attn_fwd_kernel<D><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
+  attn::attn_fwd_kernel<D, QK8><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
   return launch_status();
 }
 
@@ -552,6 +568,61 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return launch_attn_2sm(q, k, v, rows, H, prm, lens, cu_seqlens_dev == nullptr, st);
   if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
   return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+}
+
+int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, float* lse,
+                     int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                     const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                     float softmax_scale, float q_scale, float k_scale, void* stream) {
+  if (!q8 || !k8 || !v || !o) return DIT_ERR_NULL;
+  if (rows <= 0 || H <= 0 || H > 65535 || d != 128) return DIT_ERR_SHAPE;
+  if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
+  if (!(q_scale > 0.f) || !(k_scale > 0.f) || !std::isfinite(q_scale) || !std::isfinite(k_scale))
+    return DIT_ERR_SHAPE;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return DIT_ERR_ALIGN;
+  std::vector<int64_t> lens;
+  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
+  if (int s = check_device()) return s;
+  auto st = static_cast<cudaStream_t>(stream);
+  attn::Params prm{};
+  prm.cu_seqlens = cu_seqlens_dev;
+  prm.n_seq = n_seq;
+  prm.H = H;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  prm.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.force_timeout = g_force_timeout;
+  int64_t n_work = 0;
+  if (cu_seqlens_dev == nullptr) {
+    prm.dense_len = rows / n_seq;
+    prm.pairs_per_dense_seq =
+        static_cast<int32_t>((prm.dense_len + 2 * attn::kTileM - 1) / (2 * attn::kTileM));
+    n_work = static_cast<int64_t>(prm.pairs_per_dense_seq) * n_seq;
+  } else {
+    for (int64_t L : lens) n_work += (L + 2 * attn::kTileM - 1) / (2 * attn::kTileM);
+  }
+  if (n_work == 0) return DIT_OK;
+  if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
+  return launch_attn<128, true>(q8, k8, v, rows, H, prm, static_cast<int>(n_work), st);
+}
+
+int dit_quantize_e4m3(const void* x, void* out8, int64_t n, float inv_scale, void* stream) {
+  if (!x || !out8) return DIT_ERR_NULL;
+  if (n < 0 || (n % 8) != 0 || !std::isfinite(inv_scale)) return DIT_ERR_SHAPE;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(out8) & 7u)) return DIT_ERR_ALIGN;
+  if (int s = check_device()) return s;
+  if (n == 0) return DIT_OK;
+  const int64_t n8 = n / 8;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, static_cast<int64_t>(sms > 0 ? sms : 148) * 8);
+  quantize_e4m3_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(x), static_cast<uint2*>(out8), n8, inv_scale);
+  return launch_status();
 }
 
 int dit_check_device(void* stream) {

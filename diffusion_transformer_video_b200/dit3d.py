@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
 
 # every symbol include/dit3d.h declares
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_linear",
-           "dit_set_linear_variant",
+           "dit_set_linear_variant", "dit_attn_fwd_qk8", "dit_quantize_e4m3",
            "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout")
@@ -63,6 +63,8 @@ def lib():
         L.dit_gated_residual.argtypes = [P, P, P, P, i64, i32, i64, P]
         L.dit_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64, P]
         L.dit_linear.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64, P]
+        L.dit_attn_fwd_qk8.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32, f32, f32, P]
+        L.dit_quantize_e4m3.argtypes = [P, P, i64, f32, P]
         L.dit_rope3d_qk.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
                                     ctypes.POINTER(RopeDesc), P]
         L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
@@ -227,6 +229,41 @@ def dit_attn_fwd(q, k, v, n_seq=1, cu_seqlens=None, rope: RopeDesc | None = None
     _check(lib().dit_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), rows, H, d, n,
                               _ptr(cu_dev), _ptr(cu_host), float(softmax_scale),
                               ctypes.byref(rope) if rope is not None else None, _stream()))
+    _keep(cu_dev)
+    return (out, lse) if return_lse else out
+
+
+def _u8(t: torch.Tensor, name: str):
+    if not (isinstance(t, torch.Tensor) and t.dtype == torch.uint8 and t.is_cuda and t.is_contiguous()):
+        raise TypeError(f"{name} must be a contiguous uint8 (E4M3 codes) CUDA tensor")
+
+
+def dit_quantize_e4m3(x, inv_scale: float, out=None):
+    """E4M3 codes of x * inv_scale (x bf16 CUDA tensor, numel % 8 == 0) as uint8."""
+    _bf16(x, "x")
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
+    _u8(out, "out")
+    _check(lib().dit_quantize_e4m3(_ptr(x), _ptr(out), x.numel(), float(inv_scale), _stream()))
+    return out
+
+
+def dit_attn_fwd_qk8(q8, k8, v, q_scale: float, k_scale: float, n_seq=1, cu_seqlens=None,
+                     softmax_scale=0.0, out=None, return_lse=False):
+    """Attention with an E4M3 Q K^T: q8, k8 [rows, H, 128] uint8 codes standing for
+    q_scale * q8 and k_scale * k8; v bf16. Returns o (and lse)."""
+    _u8(q8, "q8")
+    _u8(k8, "k8")
+    _bf16(v, "v")
+    rows, H, d = v.shape
+    if q8.shape != v.shape or k8.shape != v.shape:
+        raise ValueError("q8, k8 and v must have the same [rows, H, d] shape")
+    out = torch.empty_like(v) if out is None else out
+    lse = torch.empty((rows, H), dtype=torch.float32, device=v.device) if return_lse else None
+    cu_dev, cu_host, ns = _cu_args(cu_seqlens)
+    n = ns if ns is not None else n_seq
+    _check(lib().dit_attn_fwd_qk8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(out), _ptr(lse), rows, H, d, n,
+                                  _ptr(cu_dev), _ptr(cu_host), float(softmax_scale),
+                                  float(q_scale), float(k_scale), _stream()))
     _keep(cu_dev)
     return (out, lse) if return_lse else out
 

@@ -189,6 +189,28 @@ int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, f
                          const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                          float softmax_scale, const dit_rope3d_desc* rope, void* stream);
 
+/* Attention whose Q K^T product runs on FP8 E4M3 operands (DiT page, "Engenharia de
+ * inferencia e paralelismo de contexto: Ulysses, Ring Attention e FP8": E4M3/E5M2
+ * activations). q8, k8: [rows, H, 128] E4M3 codes (one byte each, already rotated by
+ * 3D-RoPE where wanted) standing for q_scale * q8 and k_scale * k8; v, o: [rows, H, 128]
+ * bf16. Scores are softmax_scale * q_scale * k_scale * (q8 . k8) accumulated in fp32;
+ * P and V stay bf16, exactly as in dit_attn_fwd. Sequences, lse and stream as in
+ * dit_attn_fwd; no in-kernel RoPE. head_dim must be 128.
+ * Errors: as dit_attn_fwd; DIT_ERR_SHAPE for d != 128 or a scale that is not finite
+ * and positive. */
+int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, float* lse,
+                     int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                     const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                     float softmax_scale, float q_scale, float k_scale, void* stream);
+
+/* out8[i] = e4m3(x[i] * inv_scale): FP8 E4M3 codes of bf16 values, rounded to nearest
+ * even and saturated at +-448 (same page and section). x: n bf16 (16-byte aligned),
+ * out8: n bytes (8-byte aligned), n % 8 == 0. With inv_scale a power of two the
+ * product is exact, so every code is the nearest E4M3 value of x * inv_scale.
+ * Errors: DIT_ERR_NULL, DIT_ERR_SHAPE (n < 0, n % 8, inv_scale not finite),
+ * DIT_ERR_ALIGN. n == 0 is a no-op. */
+int dit_quantize_e4m3(const void* x, void* out8, int64_t n, float inv_scale, void* stream);
+
 /* Waits for `stream`, then reads and clears the library's device error word.
  * Returns DIT_ERR_TIMEOUT if any kernel gave up a bounded wait since the last
  * check (its outputs are then invalid), DIT_ERR_LAUNCH on a CUDA error, else DIT_OK. */
