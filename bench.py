@@ -373,7 +373,25 @@ def main():
         fp8 = {"ms": t_a8, "TFLOP/s": w.attn_flops() / (t_a8 * 1e-3) / 1e12,
                "quantize_ms": t_q8, "max_abs_vs_bf16_attention": float((o8.float() - o.float()).abs().max()),
                "in_step": False, "note": "E4M3 q, k (scale 1/64), bf16 P and V"}
-        del q8, k8, o8
+        # all of q, k, v (and P) in E4M3
+        v8 = dit3d.dit_quantize_e4m3(dev["v"], 64.0)
+        for _ in range(2):
+            dit3d.dit_attn_fwd_fp8(q8, k8, v8, 1 / 64, 1 / 64, 1 / 64, n_seq=w.n_seq,
+                                   cu_seqlens=cu, out=o8)
+        ev4 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(max(K, 3))]
+        for a, b in ev4:
+            a.record(stream)
+            dit3d.dit_attn_fwd_fp8(q8, k8, v8, 1 / 64, 1 / 64, 1 / 64, n_seq=w.n_seq,
+                                   cu_seqlens=cu, out=o8)
+            b.record(stream)
+        torch.cuda.synchronize()
+        dit3d.dit_check_device()
+        t_f8 = statistics.mean(a.elapsed_time(b) for a, b in ev4)
+        fp8["all_fp8"] = {"ms": t_f8, "TFLOP/s": w.attn_flops() / (t_f8 * 1e-3) / 1e12,
+                          "max_abs_vs_bf16_attention": float((o8.float() - o.float()).abs().max()),
+                          "note": "E4M3 q, k, v and P"}
+        del q8, k8, v8, o8
 
     # the block's linear layers (projections with the fused adaLN-Zero gate, MLP up with
     # GELU), timed on their own: not part of the step; cuBLAS on the same shapes for context

@@ -39,6 +39,7 @@
 // in-flight copies and MMAs, frees its tensor memory and exits.
 #pragma once
 #include "common.cuh"
+#include "quant.cuh"
 #include "rope3d.cuh"
 #include "sm100_ptx.cuh"
 
@@ -71,6 +72,7 @@ struct Params {
   int32_t use_rope;
   RopeParams rope;
   int32_t force_timeout;
+  float o_scale;              // multiplies O in the epilogue (V's dequantisation scale; 1 else)
 };
 
 template <int D>
@@ -213,18 +215,24 @@ __device__ __forceinline__ void rope_tile_global(uint8_t* tile, int64_t row0, in
   }
 }
 
-// QK8: q and k arrive as FP8 E4M3 codes (one byte per element, d = 128: one 128-byte
-// swizzle row per token) and S = Q K^T runs as kind::f8f6f4 MMAs (K = 32 each); the
-// host folds the two dequantisation scales into the softmax scale. P and V stay bf16.
-// The tiles keep the bf16 layout's shared-memory slots (half of each is used).
-template <int D, bool QK8 = false>
+// F8 = 1: q and k arrive as FP8 E4M3 codes (one byte per element, d = 128: one
+// 128-byte swizzle row per token) and S = Q K^T runs as kind::f8f6f4 MMAs (K = 32
+// each); the host folds the two dequantisation scales into the softmax scale; P and V
+// stay bf16. F8 = 2: v is E4M3 too (an MN-major B operand) and P is packed as E4M3
+// (4 per TMEM column; P <= 2^8 under the lazy maximum, inside E4M3's range), so
+// O += P V also runs on kind::f8f6f4; V's scale multiplies O in the epilogue. The
+// tiles keep the bf16 layout's shared-memory slots (half of each is used).
+template <int D, int F8 = 0>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using L = Smem<D>;
-  static_assert(!QK8 || D == 128, "E4M3 Q/K tiles use 128-byte rows (head_dim 128)");
+  constexpr bool QK8 = F8 >= 1, PV8 = F8 == 2;
+  static_assert(!QK8 || D == 128, "E4M3 tiles use 128-byte rows (head_dim 128)");
   constexpr int kQKBoxes = QK8 ? 1 : D / 64;                       // TMA boxes per Q/K tile
   constexpr uint32_t kQKBytes = QK8 ? kTileM * D : L::kTile;       // bytes per Q/K tile
+  constexpr int kVBoxes = PV8 ? 1 : D / 64;
+  constexpr uint32_t kVBytes = PV8 ? kTileN * D : L::kTile;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -368,7 +376,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m, -m);
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        // P for 32 keys -> 16 packed columns, stored as soon as they are ready
+        // P for 32 keys -> 16 packed bf16 columns (8 E4M3 columns), stored as soon as
+        // they are ready
         uint32_t pw[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -377,9 +386,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           f2_unpack(t2, t0, t1);
           const float e0 = ex2(t0), e1 = ex2(t1);
           l2 = f2_add(l2, f2_pack(e0, e1));
-          pw[c] = pack_bf16x2(e0, e1);
+          if constexpr (PV8) {
+            const uint32_t h = e4m3x2(e0, e1);
+            pw[c >> 1] = (c & 1) ? (pw[c >> 1] | (h << 16)) : h;
+          } else {
+            pw[c] = pack_bf16x2(e0, e1);
+          }
         }
-        ptx::tmem_st16(tS + 16 * q4, pw);
+        if constexpr (PV8) ptx::tmem_st8(tS + 8 * q4, pw);
+        else ptx::tmem_st16(tS + 16 * q4, pw);
         if (q4 == 1) {
           // keys 0-63 are in TMEM: the MMA warp may start O += P V on them
           ptx::tmem_wait_st();
@@ -399,7 +414,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float l_lo, l_hi;
       f2_unpack(l2, l_lo, l_hi);
       const float l = l_lo + l_hi;
-      const float inv_l = 1.f / l;
+      const float inv_l = p.o_scale / l;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
                       ((seq_start + row_in_seq) * p.H + head) * static_cast<int64_t>(D) * 2;
 #pragma unroll 1
@@ -453,8 +468,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             break;
           const int y = static_cast<int>(seq_start + static_cast<int64_t>(j) * kTileN);
           const uint32_t f = ptx::smem_u32(&full[st]);
-          ptx::mbar_arrive_expect_tx(f, is_k ? kQKBytes : L::kTile);
-          const int boxes = is_k ? kQKBoxes : D / 64;
+          ptx::mbar_arrive_expect_tx(f, is_k ? kQKBytes : kVBytes);
+          const int boxes = is_k ? kQKBoxes : kVBoxes;
           for (int blk = 0; blk < boxes; ++blk)
             ptx::tma_load_2d(ptx::smem_u32(smem + ring + st * L::kTile + blk * 16384), tm,
                              x0 + blk * 64, y, f);
@@ -501,12 +516,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // O_qi (+)= P_qi V over keys [64 * half, 64 * half + 64)
       auto pv = [&](int qi, int st, bool acc, int half) {
         const uint32_t va = sbase + L::kV + st * L::kTile;
+        if constexpr (PV8) {
+          // 32 keys per MMA: 8 TMEM columns of E4M3 P, 32 V rows of 128 bytes
+          constexpr uint32_t idesc_pv8 = ptx::make_idesc_e4m3_f32_bmn(kTileM, D);
 #pragma unroll
-        for (int k4 = 0; k4 < kTileN / 32; ++k4) {
-          const int kk = half * (kTileN / 32) + k4;
-          ptx::umma_ts(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
-                       ptx::make_smem_desc(va + kk * 2048, 16384, 1024, ptx::kSwizzle128B),
-                       idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          for (int k2 = 0; k2 < kTileN / 64; ++k2) {
+            const int kk = half * (kTileN / 64) + k2;
+            ptx::umma_ts_f8(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
+                            ptx::make_smem_desc(va + kk * 4096, 16384, 1024, ptx::kSwizzle128B),
+                            idesc_pv8, (acc || kk > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int k4 = 0; k4 < kTileN / 32; ++k4) {
+            const int kk = half * (kTileN / 32) + k4;
+            ptx::umma_ts(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
+                         ptx::make_smem_desc(va + kk * 2048, 16384, 1024, ptx::kSwizzle128B),
+                         idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          }
         }
       };
       // both halves, the second once the softmax has stored all of P

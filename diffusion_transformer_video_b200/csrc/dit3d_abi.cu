@@ -236,27 +236,29 @@ bool make_tmap8(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool QK8 = false>
+// F8: 0 all bf16; 1 E4M3 q and k; 2 E4M3 q, k and v (see attn_fwd_kernel)
+template <int D, int F8 = 0>
 int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32_t H,
                 const attn::Params& prm, int n_work, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   const int64_t cols = static_cast<int64_t>(H) * D;
-  const bool ok_qk = QK8 ? (make_tmap8(&tq, q, rows, cols) && make_tmap8(&tk, k, rows, cols))
-                         : (make_tmap(&tq, q, rows, cols) && make_tmap(&tk, k, rows, cols));
-  if (!ok_qk || !make_tmap(&tv, v, rows, cols)) return DIT_ERR_LAUNCH;
+  const bool ok_qk = F8 >= 1 ? (make_tmap8(&tq, q, rows, cols) && make_tmap8(&tk, k, rows, cols))
+                             : (make_tmap(&tq, q, rows, cols) && make_tmap(&tk, k, rows, cols));
+  const bool ok_v = F8 == 2 ? make_tmap8(&tv, v, rows, cols) : make_tmap(&tv, v, rows, cols);
+  if (!ok_qk || !ok_v) return DIT_ERR_LAUNCH;
   constexpr uint32_t smem = attn::Smem<D>::kRequest;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(attn::attn_fwd_kernel<D, QK8>,
+    if (cudaFuncSetAttribute(attn::attn_fwd_kernel<D, F8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return DIT_ERR_LAUNCH;
     attr_set[dev] = true;
   }
   dim3 grid(n_work, H);
-  attn::attn_fwd_kernel<D, QK8><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
+  attn::attn_fwd_kernel<D, F8><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
   return launch_status();
 }
 
@@ -550,6 +552,7 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.force_timeout = g_force_timeout;
+  prm.o_scale = 1.f;
   int64_t n_work = 0;
   if (cu_seqlens_dev == nullptr) {
     prm.dense_len = rows / n_seq;
@@ -570,15 +573,18 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
 }
 
-int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, float* lse,
-                     int64_t rows, int32_t H, int32_t d, int32_t n_seq,
-                     const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
-                     float softmax_scale, float q_scale, float k_scale, void* stream) {
+}  // extern "C"
+
+namespace {
+int attn_fp8_impl(const void* q8, const void* k8, const void* v, void* o, float* lse, int64_t rows,
+                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                  const int32_t* cu_seqlens_host, float softmax_scale, float q_scale,
+                  float k_scale, float v_scale, bool v8, void* stream) {
   if (!q8 || !k8 || !v || !o) return DIT_ERR_NULL;
   if (rows <= 0 || H <= 0 || H > 65535 || d != 128) return DIT_ERR_SHAPE;
   if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
-  if (!(q_scale > 0.f) || !(k_scale > 0.f) || !std::isfinite(q_scale) || !std::isfinite(k_scale))
-    return DIT_ERR_SHAPE;
+  for (float sc : {q_scale, k_scale, v_scale})
+    if (!(sc > 0.f) || !std::isfinite(sc)) return DIT_ERR_SHAPE;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return DIT_ERR_ALIGN;
@@ -595,6 +601,7 @@ int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, flo
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.force_timeout = g_force_timeout;
+  prm.o_scale = v8 ? v_scale : 1.f;
   int64_t n_work = 0;
   if (cu_seqlens_dev == nullptr) {
     prm.dense_len = rows / n_seq;
@@ -606,7 +613,28 @@ int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, flo
   }
   if (n_work == 0) return DIT_OK;
   if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
-  return launch_attn<128, true>(q8, k8, v, rows, H, prm, static_cast<int>(n_work), st);
+  return v8 ? launch_attn<128, 2>(q8, k8, v, rows, H, prm, static_cast<int>(n_work), st)
+            : launch_attn<128, 1>(q8, k8, v, rows, H, prm, static_cast<int>(n_work), st);
+}
+}  // namespace
+
+extern "C" {
+
+int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, float* lse,
+                     int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                     const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                     float softmax_scale, float q_scale, float k_scale, void* stream) {
+  return attn_fp8_impl(q8, k8, v, o, lse, rows, H, d, n_seq, cu_seqlens_dev, cu_seqlens_host,
+                       softmax_scale, q_scale, k_scale, 1.f, false, stream);
+}
+
+int dit_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse,
+                     int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                     const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                     float softmax_scale, float q_scale, float k_scale, float v_scale,
+                     void* stream) {
+  return attn_fp8_impl(q8, k8, v8, o, lse, rows, H, d, n_seq, cu_seqlens_dev, cu_seqlens_host,
+                       softmax_scale, q_scale, k_scale, v_scale, true, stream);
 }
 
 int dit_quantize_e4m3(const void* x, void* out8, int64_t n, float inv_scale, void* stream) {
@@ -716,6 +744,7 @@ extern "C" int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v,
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.force_timeout = g_force_timeout;
+  prm.o_scale = 1.f;
   int64_t n_work = 0;
   if (cu_seqlens_dev == nullptr) {
     prm.dense_len = rows / n_seq;

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
 
 # every symbol include/dit3d.h declares
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_linear",
-           "dit_set_linear_variant", "dit_attn_fwd_qk8", "dit_quantize_e4m3",
+           "dit_set_linear_variant", "dit_attn_fwd_qk8", "dit_attn_fwd_fp8", "dit_quantize_e4m3",
            "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout")
@@ -65,6 +65,7 @@ def lib():
         L.dit_linear.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64, P]
         L.dit_attn_fwd_qk8.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32, f32, f32, P]
         L.dit_quantize_e4m3.argtypes = [P, P, i64, f32, P]
+        L.dit_attn_fwd_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32, f32, f32, f32, P]
         L.dit_rope3d_qk.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
                                     ctypes.POINTER(RopeDesc), P]
         L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
@@ -264,6 +265,27 @@ def dit_attn_fwd_qk8(q8, k8, v, q_scale: float, k_scale: float, n_seq=1, cu_seql
     _check(lib().dit_attn_fwd_qk8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(out), _ptr(lse), rows, H, d, n,
                                   _ptr(cu_dev), _ptr(cu_host), float(softmax_scale),
                                   float(q_scale), float(k_scale), _stream()))
+    _keep(cu_dev)
+    return (out, lse) if return_lse else out
+
+
+def dit_attn_fwd_fp8(q8, k8, v8, q_scale: float, k_scale: float, v_scale: float, n_seq=1,
+                     cu_seqlens=None, softmax_scale=0.0, out=None, return_lse=False):
+    """Attention with E4M3 q, k and v ([rows, H, 128] uint8 codes standing for
+    scale * code); P rounded to E4M3 for the P V product. Returns bf16 o (and lse)."""
+    for t, n in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _u8(t, n)
+    rows, H, d = q8.shape
+    if k8.shape != q8.shape or v8.shape != q8.shape:
+        raise ValueError("q8, k8 and v8 must have the same [rows, H, d] shape")
+    out = torch.empty(rows, H, d, dtype=torch.bfloat16, device=q8.device) if out is None else out
+    _bf16(out, "out")
+    lse = torch.empty((rows, H), dtype=torch.float32, device=q8.device) if return_lse else None
+    cu_dev, cu_host, ns = _cu_args(cu_seqlens)
+    n = ns if ns is not None else n_seq
+    _check(lib().dit_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), rows, H, d, n,
+                                  _ptr(cu_dev), _ptr(cu_host), float(softmax_scale),
+                                  float(q_scale), float(k_scale), float(v_scale), _stream()))
     _keep(cu_dev)
     return (out, lse) if return_lse else out
 

@@ -209,6 +209,17 @@ int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, flo
  * product is exact, so every code is the nearest E4M3 value of x * inv_scale.
  * Errors: DIT_ERR_NULL, DIT_ERR_SHAPE (n < 0, n % 8, inv_scale not finite),
  * DIT_ERR_ALIGN. n == 0 is a no-op. */
+/* Attention with E4M3 q, k and v (same page and section): S = q_scale k_scale (q8 . k8)
+ * and O = v_scale (P8 . v8) / l both run as kind::f8f6f4 MMAs, with P rounded to E4M3
+ * (P <= 2^8 by the lazy running maximum, inside E4M3's range) and the row sum l
+ * accumulated from the unrounded fp32 P. q8, k8, v8: [rows, H, 128] E4M3 codes; o:
+ * [rows, H, 128] bf16. Other arguments and errors as dit_attn_fwd_qk8. */
+int dit_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, float* lse,
+                     int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                     const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                     float softmax_scale, float q_scale, float k_scale, float v_scale,
+                     void* stream);
+
 int dit_quantize_e4m3(const void* x, void* out8, int64_t n, float inv_scale, void* stream);
 
 /* Waits for `stream`, then reads and clears the library's device error word.

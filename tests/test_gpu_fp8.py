@@ -78,3 +78,40 @@ def test_attn_qk8_errors():
     with pytest.raises(dit3d.DitError) as e:
         dit3d.dit_attn_fwd_qk8(c, c, v, 0.0, 1.0)
     assert e.value.status == 2
+
+
+# E4M3 P in the P V product: each probability is rounded to 3 mantissa bits (relative
+# error up to 2^-4, about 2^-4/sqrt(3) rms); over N_eff keys of similar weight the output
+# error averages to ~2^-4/sqrt(3) * rms(v) / sqrt(N_eff). With >= 300 keys and unit-normal
+# v that is <= 2.1e-3 rms, so the bounds below leave about 4 sigma for the maximum.
+FP8_MAX, FP8_MEAN = 3e-2, 4e-3
+
+
+@pytest.mark.parametrize("lens,varlen", [([300], False), ([700, 700], False),
+                                         ([330, 512, 400], True), ([1], False)])
+def test_attn_fp8_parity(lens, varlen):
+    q, k, v, cu = _qk8_case(lens, 2, seed=len(lens) * 11 + lens[0])
+    inv = 64.0
+    q8, k8, v8 = (dit3d.dit_quantize_e4m3(to_dev(t), inv) for t in (q, k, v))
+    o, lse = dit3d.dit_attn_fwd_fp8(q8, k8, v8, 1 / inv, 1 / inv, 1 / inv,
+                                    n_seq=1 if varlen else len(lens),
+                                    cu_seqlens=cu if varlen else None, return_lse=True)
+    dit3d.dit_check_device()
+    v_q = oracle.quantize_e4m3(f64(v), inv) / inv
+    ref_o, ref_lse = oracle.attn_fwd_qk8(f64(q), f64(k), v_q, cu, 1 / inv, 1 / inv)
+    err = np.abs(from_dev(o) - ref_o)
+    assert np.isfinite(err).all()
+    assert err.max() <= FP8_MAX and err.mean() <= FP8_MEAN, (err.max(), err.mean())
+    # the scores are E4M3 but exact in fp32 accumulation: the LSE keeps the QK8 bound
+    np.testing.assert_allclose(lse.cpu().double().numpy(), ref_lse, atol=2e-2)
+
+
+def test_attn_fp8_single_key_is_exact_v():
+    # one key: P = 1 exactly in E4M3, so O is v's dequantised value rounded to bf16
+    q, k, v, cu = _qk8_case([1], 3, seed=9)
+    inv = 64.0
+    q8, k8, v8 = (dit3d.dit_quantize_e4m3(to_dev(t), inv) for t in (q, k, v))
+    o = dit3d.dit_attn_fwd_fp8(q8, k8, v8, 1 / inv, 1 / inv, 1 / inv)
+    dit3d.dit_check_device()
+    v_q = oracle.quantize_e4m3(f64(v), inv) / inv
+    np.testing.assert_array_equal(from_dev(o), oracle.round_bf16(v_q))
