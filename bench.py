@@ -39,7 +39,7 @@ UNIT = "TFLOP/s"
 # ("prepass" and "none" run the same kernel, without in-kernel RoPE). Heads are
 # independent, so a launch's traffic is this times its head count. None where the
 # current kernel has not been captured; other workloads report null.
-ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 528.162816e6 / 16, "none": 528.162816e6 / 16,
+ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 526.166784e6 / 16, "none": 526.166784e6 / 16,
                                  "fused": None}
 
 

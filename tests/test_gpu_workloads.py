@@ -120,3 +120,36 @@ def test_workload_linear_sampled_and_euler(case):
     dit3d.dit_check_device()
     ref = oracle.flow_euler_step(f64(inp["x"]), f64(inp["y"]), dt.astype(np.float64), frame)
     check_modulation(from_dev(xn), ref, f"{w.name} euler step")
+
+
+def test_workload_fp8_attention_sampled(case):
+    # the FP8 modes at full size, operands rotated by the RoPE pass as the bench runs them
+    w, inp = case
+    if w.head_dim != 128:
+        pytest.skip("the E4M3 attention modes take head_dim 128")
+    from tests.test_gpu_fp8 import FP8_MAX, FP8_MEAN
+    desc = dit3d.rope_desc(w.grid_h, w.grid_w, w.bands, w.base)
+    cu = w.cu_seqlens
+    cu_arg = cu if w.varlen else None
+    qr, kr = dit3d.dit_rope3d_qk(to_dev(inp["q"]), to_dev(inp["k"]), desc, n_seq=w.n_seq,
+                                 cu_seqlens=cu_arg)
+    inv = 64.0
+    q8, k8 = dit3d.dit_quantize_e4m3(qr, inv), dit3d.dit_quantize_e4m3(kr, inv)
+    v = to_dev(inp["v"])
+    v8 = dit3d.dit_quantize_e4m3(v, inv)
+    o_qk8 = dit3d.dit_attn_fwd_qk8(q8, k8, v, 1 / inv, 1 / inv, n_seq=w.n_seq, cu_seqlens=cu_arg)
+    o_fp8 = dit3d.dit_attn_fwd_fp8(q8, k8, v8, 1 / inv, 1 / inv, 1 / inv, n_seq=w.n_seq,
+                                   cu_seqlens=cu_arg)
+    dit3d.dit_check_device()
+    del q8, k8, v8, qr, kr
+    rows = wl.sample_rows(w, per_seq=32)
+    idx = torch.from_numpy(rows).cuda()
+    rope_kw = w.rope_desc()
+    ref, _ = oracle.attn_fwd_qk8(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), cu, 1 / inv,
+                                 1 / inv, qrows=rows, rope=rope_kw)
+    check_attention(from_dev(o_qk8[idx]), ref, f"{w.name} qk8 attention")
+    v_q = oracle.quantize_e4m3(f64(inp["v"]), inv) / inv
+    ref8, _ = oracle.attn_fwd_qk8(f64(inp["q"]), f64(inp["k"]), v_q, cu, 1 / inv, 1 / inv,
+                                  qrows=rows, rope=rope_kw)
+    err = np.abs(from_dev(o_fp8[idx]) - ref8)
+    assert err.max() <= FP8_MAX and err.mean() <= FP8_MEAN, (w.name, err.max(), err.mean())
