@@ -1,4 +1,5 @@
-// Flash-style forward attention with fused 3D-RoPE for sm_100a.
+// Flash-style forward attention for sm_100a, with optional in-kernel 3D-RoPE and
+// optional FP8 (E4M3) operands (template mode F8, described at the kernel).
 //
 //   o = softmax(q_rot k_rot^T * scale) v     per (sequence, head), non-causal
 //

@@ -8,6 +8,8 @@
  *   out = x + alpha_g * y                                     dit_gated_residual
  *   x  += dt_frame * u   (sampler step, not in the block)       dit_flow_euler_step
  *   out = res + alpha_g * act(x w^T + b)  (projections, MLP)     dit_linear
+ *   o   = attention on E4M3 q, k (and v, P)                     dit_attn_fwd_qk8 / _fp8
+ *   q8  = e4m3(x * inv_scale)                                   dit_quantize_e4m3
  *
  * Formulas: "DiT, Flow Matching e 3D Attention: A Engenharia de Video com IA",
  * sections "A ruptura da U-Net" (adaLN-Zero) and "3D-RoPE e atencao
