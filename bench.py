@@ -438,6 +438,25 @@ def main():
             lin[name] = {"ms": ms, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "shape": [rows, n_out, k_in],
                          "frac_burst": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
                          "cublas_ms": ms_cublas, "in_step": False}
+            if name == "linear_qkv":
+                # the same projection on E4M3 activations and weights (scales 1/16, 1/256)
+                x8 = dit3d.dit_quantize_e4m3(xin, 16.0)
+                w8 = dit3d.dit_quantize_e4m3(wt, 256.0)
+                run8 = lambda: dit3d.dit_linear_fp8(x8, w8, 1 / 16, 1 / 256, out=y)
+                for _ in range(2):
+                    run8()
+                q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                q0.record(stream)
+                for _ in range(5):
+                    run8()
+                q1.record(stream)
+                torch.cuda.synchronize()
+                dit3d.dit_check_device()
+                ms8 = q0.elapsed_time(q1) / 5
+                lin["linear_qkv_fp8"] = {"ms": ms8, "TFLOP/s": fl / (ms8 * 1e-3) / 1e12,
+                                         "shape": [rows, n_out, k_in], "in_step": False,
+                                         "note": "E4M3 x and w, fp32 accumulation, bf16 out"}
+                del x8, w8
             if name == "linear_mlp_up_gelu":
                 h_act = y  # the MLP's hidden activations feed the down projection
             del wt, y

@@ -426,11 +426,13 @@ int dit_flow_euler_step(const void* x, const void* u, const float* dt, void* out
   return launch_status();
 }
 
-int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_t M, int32_t N,
-               int32_t K, int32_t activation, const void* residual, const void* alpha,
-               int64_t rows_per_group, void* stream) {
+}  // extern "C"
+
+static int linear_impl(const void* x, const void* w, const void* bias, void* out, int64_t M, int32_t N,
+                       int32_t K, int32_t activation, const void* residual, const void* alpha,
+                       int64_t rows_per_group, bool f8, float acc_scale, void* stream) {
   if (!x || !w || !out || (residual && !alpha)) return DIT_ERR_NULL;
-  if (M < 0 || M >= (int64_t(1) << 31) || N <= 0 || K <= 0 || (N % 8) || (K % 8) ||
+  if (M < 0 || M >= (int64_t(1) << 31) || N <= 0 || K <= 0 || (N % 8) || (K % (f8 ? 16 : 8)) ||
       (activation != 0 && activation != 1))
     return DIT_ERR_SHAPE;
   if (residual && (rows_per_group <= 0 || (M % rows_per_group) != 0)) return DIT_ERR_SHAPE;
@@ -441,7 +443,9 @@ int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_
   if (M == 0) return DIT_OK;
   auto st = static_cast<cudaStream_t>(stream);
   CUtensorMap ta, tb;
-  if (!make_tmap(&ta, x, M, K, lin::kBM) || !make_tmap(&tb, w, N, K, lin::kBN)) return DIT_ERR_LAUNCH;
+  const bool maps = f8 ? (make_tmap8(&ta, x, M, K, lin::kBM) && make_tmap8(&tb, w, N, K, lin::kBN))
+                       : (make_tmap(&ta, x, M, K, lin::kBM) && make_tmap(&tb, w, N, K, lin::kBN));
+  if (!maps) return DIT_ERR_LAUNCH;
   lin::Params prm{};
   prm.bias = static_cast<const __nv_bfloat16*>(bias);
   prm.res = static_cast<const __nv_bfloat16*>(residual);
@@ -454,22 +458,27 @@ int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_
   prm.rows_per_group = residual ? rows_per_group : 1;
   prm.tiles_m = static_cast<int32_t>((M + lin::kBM - 1) / lin::kBM);
   prm.tiles_n = (N + lin::kBN - 1) / lin::kBN;
-  prm.k_blocks = (K + lin::kBK - 1) / lin::kBK;
+  const int k_per_stage = f8 ? 128 : lin::kBK;
+  prm.k_blocks = (K + k_per_stage - 1) / k_per_stage;
+  prm.acc_scale = acc_scale;
   prm.force_timeout = g_force_timeout;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set[64] = {};
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(lin::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(lin::kSmemBytes)) != cudaSuccess)
-      return DIT_ERR_LAUNCH;
-    attr_set[dev] = true;
+  static bool attr_set[2][64] = {};
+  if (dev < 64 && !attr_set[f8][dev]) {
+    const cudaError_t e =
+        f8 ? cudaFuncSetAttribute(lin::linear_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(lin::kSmemBytes))
+           : cudaFuncSetAttribute(lin::linear_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(lin::kSmemBytes));
+    if (e != cudaSuccess) return DIT_ERR_LAUNCH;
+    attr_set[f8][dev] = true;
   }
   const int64_t tiles = static_cast<int64_t>(prm.tiles_m) * prm.tiles_n;
   if (tiles >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
   if (sms <= 0) sms = 148;
-  if (g_linear_variant == 1) {
+  if (g_linear_variant == 1 && !f8) {
     // CTA pairs: 256 x 256 tiles, each CTA loads 128 rows of A and of B
     CUtensorMap tb2;
     if (!make_tmap(&tb2, w, N, K, lin::kBM)) return DIT_ERR_LAUNCH;
@@ -486,8 +495,29 @@ int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_
     return launch_status();
   }
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));
-  lin::linear_kernel<<<grid, lin::kThreads, lin::kSmemBytes, st>>>(ta, tb, prm);
+  if (f8) lin::linear_kernel<true><<<grid, lin::kThreads, lin::kSmemBytes, st>>>(ta, tb, prm);
+  else lin::linear_kernel<false><<<grid, lin::kThreads, lin::kSmemBytes, st>>>(ta, tb, prm);
   return launch_status();
+}
+
+
+extern "C" {
+
+int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_t M, int32_t N,
+               int32_t K, int32_t activation, const void* residual, const void* alpha,
+               int64_t rows_per_group, void* stream) {
+  return linear_impl(x, w, bias, out, M, N, K, activation, residual, alpha, rows_per_group, false,
+                     1.f, stream);
+}
+
+int dit_linear_fp8(const void* x8, const void* w8, const void* bias, void* out, int64_t M,
+                   int32_t N, int32_t K, int32_t activation, const void* residual,
+                   const void* alpha, int64_t rows_per_group, float x_scale, float w_scale,
+                   void* stream) {
+  if (!(x_scale > 0.f) || !(w_scale > 0.f) || !std::isfinite(x_scale) || !std::isfinite(w_scale))
+    return DIT_ERR_SHAPE;
+  return linear_impl(x8, w8, bias, out, M, N, K, activation, residual, alpha, rows_per_group, true,
+                     x_scale * w_scale, stream);
 }
 
 int dit_set_linear_variant(int variant) {

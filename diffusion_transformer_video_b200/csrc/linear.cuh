@@ -50,6 +50,7 @@ struct Params {
   int64_t rows_per_group;
   int32_t tiles_m, tiles_n, k_blocks;
   int32_t force_timeout;
+  float acc_scale;             // multiplies the accumulator (x_scale * w_scale for E4M3; 1 else)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& tm, int& tn) {
@@ -78,7 +79,7 @@ __device__ __forceinline__ float gelu_tanh(float y) {
 __device__ __forceinline__ uint4 epilogue8(const float* acc, const Params& p, int64_t row, int col) {
   float y[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) y[e] = acc[e];
+  for (int e = 0; e < 8; ++e) y[e] = acc[e] * p.acc_scale;
   if (p.bias != nullptr) {
     const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + col));
     const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
@@ -113,9 +114,14 @@ __device__ __forceinline__ uint4 epilogue8(const float* acc, const Params& p, in
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// F8: x and w arrive as FP8 E4M3 codes; a stage then holds 128 elements of K per row
+// (the same 128 bytes) and each MMA is kind::f8f6f4 with K = 32; the epilogue applies
+// x_scale * w_scale before the bias.
+template <bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
               const Params p) {
+  constexpr int kKPerStage = F8 ? 128 : kBK;  // elements of K per 128-byte row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -168,8 +174,8 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
           const uint32_t f = ptx::smem_u32(&full[s]);
           const uint32_t dst = ptx::smem_u32(smem + s * kStageBytes);
           ptx::mbar_arrive_expect_tx(f, kStageBytes);
-          ptx::tma_load_2d(dst, &tm_a, kb * kBK, tm * kBM, f);
-          ptx::tma_load_2d(dst + kABytes, &tm_b, kb * kBK, tn * kBN, f);
+          ptx::tma_load_2d(dst, &tm_a, kb * kKPerStage, tm * kBM, f);
+          ptx::tma_load_2d(dst + kABytes, &tm_b, kb * kKPerStage, tn * kBN, f);
         }
       }
       // no copy may still be in flight into shared memory when the CTA exits
@@ -201,11 +207,17 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
           }
           ptx::tc_fence_after();
           const uint32_t a0 = ptx::smem_u32(smem + s * kStageBytes), b0 = a0 + kABytes;
+          // four MMAs of 32 bytes of K each (16 bf16 or 32 E4M3 elements)
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            ptx::umma_ss(acc, ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B),
-                         ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B), idesc,
-                         (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B);
+            const uint64_t db = ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B);
+            if constexpr (F8)
+              ptx::umma_ss_f8(acc, da, db, ptx::make_idesc_e4m3_f32(kBM, kBN),
+                              (kb > 0 || kk > 0) ? 1u : 0u);
+            else
+              ptx::umma_ss(acc, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
           ptx::umma_commit(ptx::smem_u32(&empty[s]));
           issued = true;
         }

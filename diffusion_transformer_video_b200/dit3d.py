@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
 
 # every symbol include/dit3d.h declares
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_linear",
+           "dit_linear_fp8",
            "dit_set_linear_variant", "dit_attn_fwd_qk8", "dit_attn_fwd_fp8", "dit_quantize_e4m3",
            "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
@@ -63,6 +64,7 @@ def lib():
         L.dit_gated_residual.argtypes = [P, P, P, P, i64, i32, i64, P]
         L.dit_flow_euler_step.argtypes = [P, P, P, P, i64, i32, i64, P]
         L.dit_linear.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64, P]
+        L.dit_linear_fp8.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P, i64, f32, f32, P]
         L.dit_attn_fwd_qk8.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32, f32, f32, P]
         L.dit_quantize_e4m3.argtypes = [P, P, i64, f32, P]
         L.dit_attn_fwd_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32, f32, f32, f32, P]
@@ -194,6 +196,28 @@ def dit_linear(x, w, bias=None, gelu=False, residual=None, alpha=None, rows_per_
     opt = lambda t: None if t is None else _ptr(t)
     _check(lib().dit_linear(_ptr(x), _ptr(w), opt(bias), _ptr(out), M, N, K, 1 if gelu else 0,
                             opt(residual), opt(alpha), int(rows_per_group), _stream()))
+    return out
+
+
+def dit_linear_fp8(x8, w8, x_scale: float, w_scale: float, bias=None, gelu=False, residual=None,
+                   alpha=None, rows_per_group=1, out=None):
+    """dit_linear on E4M3 codes: x8 [M, K], w8 [N, K] uint8 standing for x_scale * x8 and
+    w_scale * w8; bias, residual, alpha bf16; returns bf16 [M, N]."""
+    _u8(x8, "x8")
+    _u8(w8, "w8")
+    for t, n in ((bias, "bias"), (residual, "residual"), (alpha, "alpha")):
+        if t is not None:
+            _bf16(t, n)
+    M, K = x8.shape
+    N = w8.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x8.device) if out is None else out
+    _bf16(out, "out")
+    if M == 0:
+        return out
+    opt = lambda t: None if t is None else _ptr(t)
+    _check(lib().dit_linear_fp8(_ptr(x8), _ptr(w8), opt(bias), _ptr(out), M, N, K,
+                                1 if gelu else 0, opt(residual), opt(alpha), int(rows_per_group),
+                                float(x_scale), float(w_scale), _stream()))
     return out
 
 

@@ -126,6 +126,18 @@ int dit_linear(const void* x, const void* w, const void* bias, void* out, int64_
                int32_t K, int32_t activation, const void* residual, const void* alpha,
                int64_t rows_per_group, void* stream);
 
+/* dit_linear on FP8 E4M3 operands (DiT page, "Engenharia de inferencia e paralelismo
+ * de contexto: Ulysses, Ring Attention e FP8": weights and activations in FP8).
+ * x8 [M, K] and w8 [N, K] are E4M3 codes standing for x_scale * x8 and w_scale * w8;
+ * the products run as kind::f8f6f4 MMAs with fp32 accumulation, and the epilogue
+ * (x_scale * w_scale, bias, GELU, gate) and every other argument are as in
+ * dit_linear. K % 16 == 0. Errors: as dit_linear; DIT_ERR_SHAPE for a scale that is
+ * not finite and positive. */
+int dit_linear_fp8(const void* x8, const void* w8, const void* bias, void* out, int64_t M,
+                   int32_t N, int32_t K, int32_t activation, const void* residual,
+                   const void* alpha, int64_t rows_per_group, float x_scale, float w_scale,
+                   void* stream);
+
 /* Kernel form of dit_linear for later calls in this process: 0 (default) runs one
  * CTA per 128 x 256 tile, 1 CTA pairs (cta_group::2) on 256 x 256 tiles (correct, but
  * measured 2.3x slower on B200: every k-block crosses the pair through the even CTA's

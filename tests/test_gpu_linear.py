@@ -100,3 +100,40 @@ def test_linear_bounded_wait_reports_timeout(variant):
     dit3d.dit_check_device()
     ref = (x.float() @ w.float().T)
     assert (o.float() - ref).abs().max().item() < 0.5
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 208), (1000, 1024, 512), (77, 3072, 144)])
+@pytest.mark.parametrize("mode", ["plain", "bias_gelu", "gated"])
+def test_linear_fp8_parity(M, N, K, mode):
+    x, w = bits((M, K)), bits((N, K), std=K ** -0.5)
+    inv_x, inv_w = 16.0, 256.0
+    x8 = dit3d.dit_quantize_e4m3(to_dev(x), inv_x)
+    w8 = dit3d.dit_quantize_e4m3(to_dev(w), inv_w)
+    kw, ref_kw = {}, {}
+    if mode == "bias_gelu":
+        b = bits((N,), std=0.5)
+        kw, ref_kw = dict(bias=to_dev(b), gelu=True), dict(bias=f64(b), act=1)
+    elif mode == "gated":
+        rpg = next(r for r in (64, 7, 1) if M % r == 0)
+        res, alpha = bits((M, N)), bits((M // rpg, N), std=0.5)
+        kw = dict(residual=to_dev(res), alpha=to_dev(alpha), rows_per_group=rpg)
+        ref_kw = dict(res=f64(res), alpha=f64(alpha), rows_per_group=rpg)
+    out = dit3d.dit_linear_fp8(x8, w8, 1 / inv_x, 1 / inv_w, **kw)
+    dit3d.dit_check_device()
+    xd = oracle.quantize_e4m3(f64(x), inv_x) / inv_x
+    wd = oracle.quantize_e4m3(f64(w), inv_w) / inv_w
+    ref = oracle.linear(xd, wd, **ref_kw)
+    check_modulation(from_dev(out), ref, f"linear fp8 {mode} {M}x{N}x{K}")
+
+
+def test_linear_fp8_errors():
+    x8 = torch.zeros(64, 40, dtype=torch.uint8, device="cuda")
+    w8 = torch.zeros(64, 40, dtype=torch.uint8, device="cuda")
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_linear_fp8(x8, w8, 1.0, 1.0)  # K = 40 is not a multiple of 16
+    assert e.value.status == 2
+    x8 = torch.zeros(64, 64, dtype=torch.uint8, device="cuda")
+    w8 = torch.zeros(64, 64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_linear_fp8(x8, w8, -1.0, 1.0)
+    assert e.value.status == 2
