@@ -2,11 +2,15 @@
 """Benchmark of the DiT attention-block hot path on B200.
 
 One step = one pass of the whole path over one batch of the workload:
-  u   = dit_adaln_modulate(x, gamma, beta)               (adaLN, memory-bound)
-  o   = dit_attn_fwd(q, k, v, rope=3D-RoPE)              (RoPE fused, tensor-core bound)
-  out = dit_gated_residual(x, o, alpha)                  (adaLN-Zero gate, memory-bound)
-The q/k/v projections around the path are not part of it; q, k, v, x and the adaLN
-parameters are seeded synthetic bf16 tensors with the workload's shapes.
+  u        = dit_adaln_modulate(x, gamma, beta)          (adaLN, memory-bound)
+  q_r, k_r = dit_rope3d_qk(q, k, 3D-RoPE)                (RoPE pass, memory-bound)
+  o        = dit_attn_fwd(q_r, k_r, v)                   (tensor-core bound)
+  out      = dit_gated_residual(x, o, alpha)             (adaLN-Zero gate, memory-bound)
+(--rope-mode fused rotates inside the attention kernel instead.) The q/k/v
+projections around the path are not part of it; q, k, v, x and the adaLN parameters
+are seeded synthetic bf16 tensors with the workload's shapes. Timed separately and
+reported as components, not in the step: the Euler step, the block's linear layers
+(bf16 and E4M3), and the E4M3 attention modes.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p] [--impl reference]
 
