@@ -20,7 +20,10 @@
  * Conventions shared by every call
  *  - Tensors are dense, row-major, token-major bf16 in device memory, with no
  *    strides: activations [rows, D]; q/k/v/o [rows, H, d] (= [rows, D], D = H*d).
- *  - Every device pointer must be 16-byte aligned (128-bit loads and TMA).
+ *    The FP8 calls take the same layouts with one E4M3 code (byte) per element.
+ *  - Every tensor pointer must be 16-byte aligned (128-bit loads and TMA); the
+ *    exceptions are stated at their calls (fp32 lse and dt: 4 bytes; the codes
+ *    written by dit_quantize_e4m3: 8 bytes).
  *  - The caller owns every buffer. Calls allocate nothing per call; the RoPE
  *    cos/sin tables (fp64 on the host, stored fp32) are cached in device memory
  *    per (device, descriptor, extent) on first use and freed by dit_shutdown().
