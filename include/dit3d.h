@@ -145,7 +145,8 @@ int dit_linear_fp8(const void* x8, const void* w8, const void* bias, void* out, 
  * CTA per 128 x 256 tile, 1 CTA pairs (cta_group::2) on 256 x 256 tiles (correct, but
  * measured 2.3x slower on B200: every k-block crosses the pair through the even CTA's
  * barriers). Same results up to the order of fp32 additions. No counterpart in the
- * source pages.
+ * source pages. A plain process-wide setting, not synchronised: set it before other
+ * threads issue calls.
  * Errors: DIT_ERR_SHAPE for any other value. */
 int dit_set_linear_variant(int variant);
 
@@ -255,6 +256,8 @@ void dit_shutdown(void);
  * 1: CTA pairs on two SMs sharing each tcgen05 MMA (cta_group::2, M = 256): each SM
  * loads and rotates half of every K tile and loads half of every V tile. Both give the
  * same results (same rounding steps); variant 0 is faster on the measured workloads.
+ * A plain process-wide setting, not synchronised: set it before other threads issue
+ * calls. The E4M3 attention calls always use variant 0.
  * Returns DIT_ERR_SHAPE for any other value. */
 int dit_set_attn_variant(int variant);
 
