@@ -170,7 +170,9 @@ int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, 
  * over the keys j of the query's own sequence (packed sequences never see one
  * another). With `rope` non-NULL, q and k are rotated by 3D-RoPE inside the
  * kernel as their tiles are loaded (fp32 rotation, bf16 operand); with NULL they
- * are used as given.
+ * are used as given. Rotating q and k first with dit_rope3d_qk and passing NULL
+ * gives the same bits and is faster on long sequences (in-kernel, every K tile is
+ * rotated again for each pair of query tiles); the in-kernel form needs no scratch.
  *   q, k, v, o : [rows, H, d] bf16, o must not overlap q, k or v
  *   lse        : NULL or [rows, H] fp32, natural-log sum of exp(scale * scores)
  *   softmax_scale <= 0 selects 1/sqrt(d).
