@@ -88,3 +88,41 @@ def lpt_assign(lengths, world: int) -> list[list[int]]:
         out[r].append(i)
         heapq.heappush(heap, (load + int(lengths[i]) ** 2, r))
     return [sorted(s) for s in out]
+
+
+def varlen_plan(cu_seqlens, world: int):
+    """Placement of a packed batch's sequences on `world` ranks (``lpt_assign``).
+
+    Returns, per rank, a dict with ``seqs`` (sequence indices), ``rows`` (the global
+    row indices of those sequences, in order, as an int64 tensor) and ``cu`` (the
+    packed prefix sums of the local batch, int32)."""
+    cu = [int(c) for c in cu_seqlens]
+    lens = [cu[i + 1] - cu[i] for i in range(len(cu) - 1)]
+    plans = []
+    for seqs in lpt_assign(lens, world):
+        rows = [torch.arange(cu[s], cu[s + 1], dtype=torch.int64) for s in seqs]
+        local_cu = [0]
+        for s in seqs:
+            local_cu.append(local_cu[-1] + lens[s])
+        plans.append({"seqs": seqs,
+                      "rows": torch.cat(rows) if rows else torch.zeros(0, dtype=torch.int64),
+                      "cu": torch.tensor(local_cu, dtype=torch.int32)})
+    return plans
+
+
+def varlen_gather(out_local: torch.Tensor, plans, total_rows: int, group=None) -> torch.Tensor:
+    """Every rank's local rows (in its plan's order) back into the full packed batch,
+    on every rank: one all_gather of row blocks padded to the longest rank."""
+    world = dist.get_world_size(group)
+    width = max(int(p["rows"].numel()) for p in plans)
+    pad = torch.zeros((width,) + tuple(out_local.shape[1:]), dtype=out_local.dtype,
+                      device=out_local.device)
+    pad[: out_local.shape[0]] = out_local
+    blocks = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(blocks, pad, group=group)
+    full = torch.empty((total_rows,) + tuple(out_local.shape[1:]), dtype=out_local.dtype,
+                       device=out_local.device)
+    for r, p in enumerate(plans):
+        n = int(p["rows"].numel())
+        full[p["rows"].to(full.device)] = blocks[r][:n]
+    return full

@@ -113,3 +113,41 @@ def test_lpt_assign_is_a_partition_within_four_thirds_of_optimal(seed):
 def test_lpt_assign_small_cases():
     assert ulysses.lpt_assign([5, 4, 3, 3], 2) == [[0, 3], [1, 2]]
     assert ulysses.lpt_assign([1, 1, 1], 4) == [[0], [1], [2], []]
+
+
+def _varlen_worker(rank, world, port, q, lens):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        N = int(cu[-1])
+        Q, K, V = _full(N, 2, 16, 9)
+        plans = ulysses.varlen_plan(cu, world)
+        mine = plans[rank]
+        idx = mine["rows"].numpy()
+        # this rank attends over its whole sequences only (the oracle stands in for the kernel)
+        o_loc, _ = oracle.attn_fwd(Q[idx], K[idx], V[idx], mine["cu"].numpy())
+        full = ulysses.varlen_gather(torch.from_numpy(np.ascontiguousarray(o_loc)), plans, N).numpy()
+        ref, _ = oracle.attn_fwd(Q, K, V, cu)
+        q.put((rank, float(np.abs(full - ref).max()), sorted(mine["seqs"])))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_varlen_sequences_placed_by_lpt_give_the_packed_result(world):
+    lens = [40, 7, 64, 1, 33, 20, 50]
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_varlen_worker, args=(r, world, port, q, lens)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    placed = sorted(s for _, _, seqs in res for s in seqs)
+    assert placed == list(range(len(lens)))                 # every sequence exactly once
+    for rank, err, _ in res:
+        assert err == 0.0, f"rank {rank}: gathered output differs from the packed batch by {err}"
