@@ -108,7 +108,7 @@ def _ptr(t):
 
 def _bf16(t: torch.Tensor, name: str):
     if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
-        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+        raise TypeError(f"{name} must be a contiguous bf16 CUDA tensor")
 
 
 def _keep(cu_dev):
