@@ -131,8 +131,9 @@ def cpu_oracle_attention(w, qkv64, n_rows: int, seed: int = 0):
     cu = w.cu_seqlens
     q, k, v = qkv64
     t0 = time.perf_counter()
-    oracle.attn_fwd(q, k, v, cu, qrows=rows, rope=w.rope_desc())
+    ref_o, _ = oracle.attn_fwd(q, k, v, cu, qrows=rows, rope=w.rope_desc())
     dt = time.perf_counter() - t0
+    cpu_oracle_attention.last = (rows, ref_o)  # kept for the parity figures of the GPU arm
     seq_of = np.searchsorted(cu, rows, side="right") - 1
     flops = float(sum(4.0 * (cu[s + 1] - cu[s]) * w.head_dim * w.heads for s in seq_of))
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
@@ -558,6 +559,12 @@ def main():
         tf, dt, sample, threads = cpu_oracle_attention(w, widen_qkv(inp), args.cpu_rows, args.seed)
         cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
                "seconds": dt}
+        # the step's attention output on the same sampled rows, against the oracle
+        s_rows, ref_o = cpu_oracle_attention.last
+        got = o[torch.from_numpy(s_rows).cuda()].float().cpu().double().numpy()
+        err = np.abs(got - ref_o)
+        cpu["parity"] = {"rows": int(len(s_rows)), "max_abs": float(err.max()),
+                         "mean_abs": float(err.mean()), "tolerance_max_mean": [2e-2, 2e-3]}
 
     if rank == 0:
         line = {
