@@ -267,6 +267,65 @@ def test_attn_qk8_is_attention_of_the_quantised_operands():
     np.testing.assert_allclose(l8, l, atol=1e-13)
 
 
+def test_attn_qk8_rope_on_a_single_frame_with_time_band_energy_is_plain_attention():
+    # T = 1: every token has t = 0, so the t band turns by nothing; q and k hold energy in
+    # the t band only, so the h and w bands rotate zeros. The rotation is then the
+    # identity, the bf16 rounding of operands already on the e4m3 grid is exact, and the
+    # E4M3 attention with RoPE must equal plain attention of the unrotated operands.
+    rng = np.random.default_rng(16)
+    gh, gw, H, d, bands = 3, 4, 2, 32, (16, 8, 8)
+    N = gh * gw
+    q = np.zeros((N, H, d))
+    k = np.zeros((N, H, d))
+    q[..., :16] = oracle.quantize_e4m3(rng.standard_normal((N, H, 16)) * 8) / 8
+    k[..., :16] = oracle.quantize_e4m3(rng.standard_normal((N, H, 16)) * 8) / 8
+    v = rng.standard_normal((N, H, d))
+    cu = np.array([0, N], np.int32)
+    rope = dict(grid_h=gh, grid_w=gw, bands=bands)
+    o8, l8 = oracle.attn_fwd_qk8(q, k, v, cu, 1 / 8, 1 / 8, rope=rope)
+    o, l = oracle.attn_fwd(q, k, v, cu)
+    np.testing.assert_allclose(o8, o, atol=1e-13)
+    np.testing.assert_allclose(l8, l, atol=1e-13)
+    # energy outside the t band does turn (w > 0 tokens): the two must then differ
+    q2 = q.copy()
+    q2[..., 16:] = 1.0
+    k2 = k.copy()
+    k2[..., 24:] = 1.0
+    o8c, _ = oracle.attn_fwd_qk8(q2, k2, v, cu, 1 / 8, 1 / 8, rope=rope)
+    oc, _ = oracle.attn_fwd(q2, k2, v, cu)
+    assert not np.allclose(o8c, oc, atol=1e-6)
+
+
+def test_attn_qk8_rope_order_rotate_round_bf16_then_e4m3_two_keys():
+    # Hand-computed case that fixes the order of the steps (DiT page, 3D-RoPE section:
+    # the scores use the rotated q and k; FP8 section: E4M3 operands; the rotated
+    # operand is a bf16 tensor before it is quantised). d = 2 with one w-band pair of
+    # frequency base^0 = 1; a 1 x 2 patch grid, so token 0 sits at w = 0 (no turn) and
+    # token 1 at w = 1 (a turn of 1 rad). q_0 = (1, 0); k_0 = (1.5, 0); k_1 = (1.96875, 0).
+    #   k_1 rotated: (1.96875 cos 1, 1.96875 sin 1) = (1.063720..., 1.656673...)
+    #   bf16:        (1.0625, 1.65625)        (bf16 spacing 2^-7 in [1, 2))
+    #   E4M3:        (1.0,    1.625)          (1.0625 is the tie between 1.0 and 1.125:
+    #                                          nearest even keeps 1.0)
+    # so with scale 1 the scores of query 0 are s_0 = 1.5 and s_1 = 1.0, and
+    #   o_0 = sigmoid(0.5) v_0 + sigmoid(-0.5) v_1,  lse_0 = log(e^1.5 + e^1.0).
+    # Skipping the bf16 rounding gives s_1 = 1.125; quantising before rotating gives
+    # s_1 = bf16(2 cos 1) = 1.078125: both fail below.
+    q = np.array([[[1.0, 0.0]], [[0.25, 0.5]]])
+    k = np.array([[[1.5, 0.0]], [[1.96875, 0.0]]])
+    v = np.array([[[1.0, 0.0]], [[0.0, 1.0]]])
+    cu = np.array([0, 2], np.int32)
+    rope = dict(grid_h=1, grid_w=2, bands=(0, 0, 2))
+    o, lse = oracle.attn_fwd_qk8(q, k, v, cu, 1.0, 1.0, scale=1.0, qrows=[0], rope=rope)
+    sig = lambda z: 1.0 / (1.0 + math.exp(-z))
+    np.testing.assert_allclose(o[0, 0], [sig(0.5), sig(-0.5)], atol=1e-15)
+    np.testing.assert_allclose(lse[0, 0], math.log(math.exp(1.5) + math.exp(1.0)), atol=1e-15)
+    # the same case with the scales moved onto the codes (q_scale = k_scale = 1/2, codes
+    # e4m3(2 x)): a power-of-two scale moves the E4M3 grid with the values, so the same
+    # values come out and the tie at 1.0625 (2.125 in code units) again keeps the even 1.0
+    o2, _ = oracle.attn_fwd_qk8(q, k, v, cu, 0.5, 0.5, scale=1.0, qrows=[0], rope=rope)
+    np.testing.assert_allclose(o2[0, 0], [sig(0.5), sig(-0.5)], atol=1e-15)
+
+
 def test_rope_preserves_norm():
     # Orthogonal rotations (DiT page, 3D-RoPE section): |R q| = |q| per head.
     gh, gw, T, H, d = 3, 5, 4, 3, 64
