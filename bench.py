@@ -221,6 +221,214 @@ def job_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> flo
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
+STEP_INPUTS = ("x", "q", "k", "v", "gamma", "beta", "alpha")
+
+
+def param_sets_on_device(w, seed, torch):
+    """The workload's adaLN parameter sets (two for the 720P expert pair) on the device."""
+    from diffusion_transformer_video_b200 import workloads as wl
+    sets = []
+    for ps in range(w.param_sets):
+        prm = wl.make_inputs(w, seed, which=("gamma", "beta", "alpha"), param_set=ps)
+        sets.append({k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda()
+                     for k, v in prm.items()})
+    return sets
+
+
+class StepRunner:
+    """One workload's step on the device: modulate -> RoPE pass -> attention -> residual,
+    with CUDA events around each call. Step i uses adaLN parameter set i % param_sets
+    (the 720P workload alternates its high- and low-noise experts)."""
+
+    def __init__(self, w, seed, args, torch, dit3d, host=None):
+        from diffusion_transformer_video_b200 import workloads as wl
+        self.w, self.args, self.torch, self.dit3d = w, args, torch, dit3d
+        if host is None:
+            inp = wl.make_inputs(w, seed, which=("x", "q", "k", "v"))
+            host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16)
+                    for k, v in inp.items()}
+        self.dev = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+        self.params = param_sets_on_device(w, seed, torch)
+        rows, D, H, d = w.rows, w.d_model, w.heads, w.head_dim
+        self.desc = dit3d.rope_desc(w.grid_h, w.grid_w, w.bands, w.base)
+        self.cu = None
+        if w.varlen:
+            cu_host = torch.from_numpy(w.cu_seqlens)
+            self.cu = (cu_host.cuda(), cu_host)
+        self.u = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+        self.o = torch.empty(rows, H, d, dtype=torch.bfloat16, device="cuda")
+        self.out = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+        self.q_rot = self.k_rot = None
+        if args.rope_mode == "prepass":
+            self.q_rot, self.k_rot = torch.empty_like(self.dev["q"]), torch.empty_like(self.dev["k"])
+        self.stream = torch.cuda.current_stream()
+
+    def step(self, b=None, i=0, ev=None, out_t=None):
+        """One pass of the path over the batch `b` (default: this workload's inputs)."""
+        w, dit3d, args = self.w, self.dit3d, self.args
+        b = self.dev if b is None else b
+        prm = b.get("params", self.params)[i % w.param_sets]
+        out_t = self.out if out_t is None else out_t
+        rec = (lambda k: ev[k].record(self.stream)) if ev is not None else (lambda k: None)
+        rec(0)
+        dit3d.dit_adaln_modulate(b["x"], prm["gamma"], prm["beta"], w.rows_per_group, out=self.u)
+        rec(1)
+        if args.rope_mode == "prepass":
+            dit3d.dit_rope3d_qk(b["q"], b["k"], self.desc, n_seq=w.n_seq, cu_seqlens=self.cu,
+                                q_out=self.q_rot, k_out=self.k_rot)
+            qa, ka = self.q_rot, self.k_rot
+        else:
+            qa, ka = b["q"], b["k"]
+        rec(2)
+        dit3d.dit_attn_fwd(qa, ka, b["v"], n_seq=w.n_seq, cu_seqlens=self.cu, out=self.o,
+                           rope=self.desc if args.rope_mode == "fused" else None)
+        rec(3)
+        dit3d.dit_gated_residual(b["x"], self.o.view(w.rows, w.d_model), prm["alpha"],
+                                 w.rows_per_group, out=out_t)
+        rec(4)
+
+    def timed(self, steps, warmup, barrier=lambda: None, local_rank=0):
+        """W untimed steps, then `steps` timed ones (L2 flushed between steps when one
+        input tensor fits in L2). Returns per-call mean times, the timed region's length
+        and the clocks sampled during it."""
+        torch = self.torch
+        for i in range(warmup):
+            self.step(i=i)
+        torch.cuda.synchronize()
+        self.dit3d.dit_check_device()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+        flush = None if l2_resident_free(self.w) else torch.empty(L2_FLUSH_BYTES // 4,
+                                                                  dtype=torch.float32,
+                                                                  device="cuda")
+        barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local_rank) as clk:
+            t_start = torch.cuda.Event(enable_timing=True)
+            t_end = torch.cuda.Event(enable_timing=True)
+            t_start.record(self.stream)
+            for i in range(steps):
+                if flush is not None:
+                    flush.fill_(float(i))
+                self.step(i=i, ev=evs[i])
+            t_end.record(self.stream)
+            torch.cuda.synchronize()
+        barrier()
+        self.dit3d.dit_check_device()
+        elapsed = (t_start.elapsed_time(t_end) if flush is None
+                   else sum(e[0].elapsed_time(e[4]) for e in evs))
+        mean = lambda a, b: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+        return {"elapsed_ms": elapsed, "mod": mean(0, 1), "rope": mean(1, 2), "attn": mean(2, 3),
+                "res": mean(3, 4), "clocks": clk.summary()}
+
+    def free(self):
+        for name in ("dev", "params", "u", "o", "out", "q_rot", "k_rot", "cu"):
+            setattr(self, name, None)
+        self.torch.cuda.empty_cache()
+
+
+def workload_figures(w, t, pk, rope_mode) -> dict:
+    """Throughput and roofline fractions of one workload's timed steps: attention TFLOP/s
+    against the burst bf16 peak (and the sustained one), memory-bound calls in GB/s
+    against the HBM copy bandwidth."""
+    rows, D = w.rows, w.d_model
+    flops = w.attn_flops()
+    att = flops / (t["attn"] * 1e-3) / 1e12
+    def mem(ms, nbytes):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "GB/s": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "bytes": nbytes}
+    out = {
+        "attn_fwd": {"ms": t["attn"], "TFLOP/s": att, "frac": att / pk["bf16_tflops"],
+                     "frac_sustained": att / pk["bf16_tflops_sustained"], "flops": flops},
+        "adaln_modulate": mem(t["mod"], 4.0 * rows * D),
+        "rope3d_qk": mem(t["rope"], 8.0 * rows * D) if rope_mode == "prepass" else None,
+        "gated_residual": mem(t["res"], 6.0 * rows * D),
+        "step_ms": t["step_ms"], "step_TFLOP/s": flops / (t["step_ms"] * 1e-3) / 1e12,
+        "rows": rows, "sequences": w.n_seq, "heads": w.heads, "d_model": D,
+        "clocks_sm_mhz": t["clocks"]["sm_mhz"], "clock_reasons": t["clocks"]["reasons"],
+    }
+    if w.param_sets > 1:
+        out["param_sets"] = f"{w.param_sets} adaLN parameter sets, alternated step by step"
+    if w.varlen:
+        out["frames"] = list(w.frames)
+        out["seqlens"] = list(w.seqlens)
+    if w.name.startswith("tiny"):
+        out["note"] = "latency-bound (64 tokens): reported, not held to the roofline targets"
+    return out
+
+
+def run_ulysses(args, rank, world, local_rank):
+    """Ulysses sequence parallelism over the job's ranks: ONE batch of the workload,
+    each sequence split over the ranks by tokens (strong scaling), head chunks whose
+    all-to-all overlaps the previous chunk's RoPE pass and attention. A step is one
+    ulysses_attention call (exchange, RoPE, attention, exchange back)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from diffusion_transformer_video_b200 import dit3d, ulysses, workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    if world == 1 and "MASTER_PORT" not in os.environ:   # a plain single-process run
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(sk.getsockname()[1]))
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local_rank))
+    try:
+        w = resolve_workload(args)
+        layout = ulysses.UlyssesLayout(w.cu_seqlens, world)
+        mine = layout.local_rows(rank).numpy()
+        inp = wl.make_inputs(w, args.seed, which=("q", "k", "v"))
+        loc = {k: torch.from_numpy(np.ascontiguousarray(v[mine]).view(np.int16))
+               .view(torch.bfloat16).cuda() for k, v in inp.items()}
+        del inp
+        desc = dit3d.rope_desc(w.grid_h, w.grid_w, w.bands, w.base)
+        h_loc = w.heads // world
+        chunks = args.head_chunks if args.head_chunks else max(
+            c for c in range(1, h_loc + 1) if h_loc % c == 0 and c <= 4)
+        run = lambda: ulysses.ulysses_attention(loc["q"], loc["k"], loc["v"], rope=desc,
+                                                cu_seqlens=w.cu_seqlens, head_chunks=chunks)
+        for _ in range(args.warmup):
+            run()
+        torch.cuda.synchronize()
+        dit3d.dit_check_device()
+        dist.barrier()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        with ClockSampler(local_rank) as clk:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        dist.barrier()
+        dit3d.dit_check_device()
+        ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dist, "cuda")[0]
+        clocks = clk.summary()
+        flops = w.attn_flops()
+        if rank == 0:
+            pk = _peaks()
+            value = flops / (ms * 1e-3) / 1e12
+            line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                    "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                    "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v)",
+                    "config": dict(workload_config(w, world),
+                                   parallelism=f"ulysses{world} (tokens split over ranks, "
+                                               f"{chunks} head chunks per rank)"),
+                    "gpu_launches": None,
+                    "roofline": {"bound": "tensor", "achieved": value / world,
+                                 "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                 "frac": value / world / pk["bf16_tflops"], "traffic": None,
+                                 "kernel": "whole Ulysses step per GPU (exchanges included)"},
+                    "clocks": clocks, "e2e": None, "cpu_baseline": None}
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -235,6 +443,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-linear", action="store_true",
                     help="skip timing the block's linear layers (separate components)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other four workloads (the `workloads` object)")
+    ap.add_argument("--workload-steps", type=int, default=10,
+                    help="timed steps per workload in the `workloads` object")
     ap.add_argument("--rope-mode", default="prepass", choices=["prepass", "fused", "none"],
                     help="prepass: dit_rope3d_qk into scratch, then attention (the product "
                          "path, fastest); fused: RoPE inside the attention kernel (no scratch); "
@@ -243,6 +455,11 @@ def main():
                     help="0: single-CTA attention kernel; 1: CTA-pair (cta_group::2) kernel")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (smaller cases for profiling)")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="Ulysses sequence parallelism: one batch split over the ranks by "
+                         "tokens (strong scaling) instead of one batch per rank")
+    ap.add_argument("--head-chunks", type=int, default=0,
+                    help="Ulysses: head chunks per rank (default: up to 4)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -252,6 +469,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.ulysses:
+        run_ulysses(args, rank, world, local_rank)
         return
 
     import torch
@@ -269,84 +489,28 @@ def main():
             dist.barrier()
 
     dit3d.dit_set_attn_variant(args.attn_variant)
+    pk = _peaks()
     w = resolve_workload(args)
     # every rank runs its own batch of the workload (seeded per rank)
     seed = rank_seed(args.seed, rank)
-    inp = wl.make_inputs(w, seed)
+    inp = wl.make_inputs(w, seed, which=("x", "q", "k", "v"))
     host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
             for k, v in inp.items()}
-    dev = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+    run = StepRunner(w, seed, args, torch, dit3d, host=host)
+    host.update({f"{k}{ps}": v.cpu().pin_memory() for ps, prm in enumerate(run.params)
+                 for k, v in prm.items()})
+    dev, stream = run.dev, run.stream
     rows, D, H, d = w.rows, w.d_model, w.heads, w.head_dim
     rpg = w.rows_per_group
-    desc = dit3d.rope_desc(w.grid_h, w.grid_w, w.bands, w.base)
-    cu = None
-    if w.varlen:
-        cu_host = torch.from_numpy(w.cu_seqlens)
-        cu = (cu_host.cuda(), cu_host)
-    u = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
-    o = torch.empty(rows, H, d, dtype=torch.bfloat16, device="cuda")
-    out = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
-    stream = torch.cuda.current_stream()
-
-    if args.rope_mode == "prepass":
-        q_rot, k_rot = torch.empty_like(dev["q"]), torch.empty_like(dev["k"])
-
-    def step(b, ev=None, out_t=None):
-        out_t = out if out_t is None else out_t
-        if ev is not None:
-            ev[0].record(stream)
-        dit3d.dit_adaln_modulate(b["x"], b["gamma"], b["beta"], rpg, out=u)
-        if ev is not None:
-            ev[1].record(stream)
-        if args.rope_mode == "prepass":
-            dit3d.dit_rope3d_qk(b["q"], b["k"], desc, n_seq=w.n_seq, cu_seqlens=cu,
-                                q_out=q_rot, k_out=k_rot)
-            qa, ka = q_rot, k_rot
-        else:
-            qa, ka = b["q"], b["k"]
-        if ev is not None:
-            ev[2].record(stream)
-        dit3d.dit_attn_fwd(qa, ka, b["v"], n_seq=w.n_seq, cu_seqlens=cu, out=o,
-                           rope=desc if args.rope_mode == "fused" else None)
-        if ev is not None:
-            ev[3].record(stream)
-        dit3d.dit_gated_residual(b["x"], o.view(rows, D), b["alpha"], rpg, out=out_t)
-        if ev is not None:
-            ev[4].record(stream)
-
-    for _ in range(args.warmup):
-        step(dev)
-    torch.cuda.synchronize()
-    dit3d.dit_check_device()
+    cu = run.cu
+    o, u = run.o, run.u
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    # inputs smaller than L2: write a buffer twice its size between steps and time the
-    # steps alone (their events), so every step starts from a cold L2
-    flush = None if l2_resident_free(w) else torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32,
-                                                        device="cuda")
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for i in range(K):
-            if flush is not None:
-                flush.fill_(float(i))
-            step(dev, evs[i])
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier()
-    dit3d.dit_check_device()
-    elapsed_ms = (t_start.elapsed_time(t_end) if flush is None
-                  else sum(e[0].elapsed_time(e[4]) for e in evs))
-    del flush
-    t_mod = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    t_rope = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    t_att = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    t_res = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
-    clocks = clk.summary()
+    t = run.timed(K, args.warmup, barrier, local_rank)
+    elapsed_ms = t["elapsed_ms"]
+    t_mod, t_rope, t_att, t_res = t["mod"], t["rope"], t["attn"], t["res"]
+    clocks = t["clocks"]
+    q_rot = run.q_rot
 
     # the sampler's Euler step (x += dt_frame * u), timed on its own: not part of the step
     frame = w.grid_h * w.grid_w
@@ -369,6 +533,7 @@ def main():
     # products), then attention with the E4M3 product; timed on its own, not in the step
     fp8 = None
     if d == 128 and args.rope_mode == "prepass":
+        k_rot = run.k_rot
         q8 = torch.empty(rows, H, d, dtype=torch.uint8, device="cuda")
         k8 = torch.empty_like(q8)
         o8 = torch.empty_like(o)
@@ -419,7 +584,6 @@ def main():
     # the block's linear layers (projections with the fused adaLN-Zero gate, MLP up with
     # GELU), timed on their own: not part of the step; cuBLAS on the same shapes for context
     lin = {}
-    pk = _peaks()
     if not args.no_linear:
         gen = torch.Generator(device="cuda").manual_seed(args.seed + 7)
         hidden = 4 * D
@@ -435,14 +599,14 @@ def main():
             kw = dict(gelu=gelu, out=y)
             if gated:
                 kw.update(residual=dev["x"], alpha=alpha_g, rows_per_group=rpg, out=x_next)
-            run = lambda: dit3d.dit_linear(xin, wt, **kw)
+            run_lin = lambda: dit3d.dit_linear(xin, wt, **kw)
             for _ in range(2):
-                run()
+                run_lin()
             pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                      for _ in range(5)]
             for a, b in pairs:
                 a.record(stream)
-                run()
+                run_lin()
                 b.record(stream)
             torch.cuda.synchronize()
             dit3d.dit_check_device()
@@ -484,16 +648,21 @@ def main():
                 h_act = y  # the MLP's hidden activations feed the down projection
             del wt, y
 
-    # end to end: every step copies its inputs from pinned host memory and its result
-    # back, through the same calls. Two device buffer sets and one upload and one
-    # download stream pipeline the steps: step i+1's inputs upload and step i-1's result
-    # downloads while step i computes (a set is reused only after the step that read it
-    # has finished, an output buffer only after its download).
-    e2e_keys = ("x", "q", "k", "v", "gamma", "beta", "alpha")
-    sets = [{k: torch.empty_like(dev[k]) for k in e2e_keys} for _ in range(2)]
+    # end to end: every step copies its inputs (x, q, k, v and the step's adaLN
+    # parameters) from pinned host memory and its result back, through the same calls.
+    # Two device buffer sets and one upload and one download stream pipeline the steps:
+    # step i+1's inputs upload and step i-1's result downloads while step i computes (a
+    # set is reused only after the step that read it has finished, an output buffer only
+    # after its download).
+    data_keys = ("x", "q", "k", "v")
+    prm_keys = ("gamma", "beta", "alpha")
+    sets = [dict({k: torch.empty_like(dev[k]) for k in data_keys},
+                 params=[{k: torch.empty_like(run.params[0][k]) for k in prm_keys}] * 1)
+            for _ in range(2)]
     outs = [torch.empty(rows, D, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     res_host = [torch.empty(rows, D, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    h2d = sum(host[k].numel() * 2 for k in e2e_keys)
+    h2d = (sum(host[k].numel() * 2 for k in data_keys)
+           + sum(run.params[0][k].numel() * 2 for k in prm_keys))
     d2h = res_host[0].numel() * 2
     up_stream, down_stream = torch.cuda.Stream(), torch.cuda.Stream()
     loaded = [torch.cuda.Event() for _ in range(2)]
@@ -506,8 +675,11 @@ def main():
         with torch.cuda.stream(up_stream):
             if i >= 2:
                 up_stream.wait_event(computed[bset])     # step i-2 has read this set
-            for k in e2e_keys:
+            for k in data_keys:
                 sets[bset][k].copy_(host[k], non_blocking=True)
+            ps = i % w.param_sets                        # this step's parameter set
+            for k in prm_keys:
+                sets[bset]["params"][0][k].copy_(host[f"{k}{ps}"], non_blocking=True)
             loaded[bset].record(up_stream)
 
     barrier()
@@ -524,7 +696,7 @@ def main():
         stream.wait_event(loaded[bset])
         if i >= 2:
             stream.wait_event(drained[bset])             # step i-2's result has left outs[bset]
-        step(sets[bset], out_t=outs[bset])
+        run.step(sets[bset], i=0, out_t=outs[bset])
         computed[bset].record(stream)
         with torch.cuda.stream(down_stream):
             down_stream.wait_event(computed[bset])
@@ -535,8 +707,11 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
-    # the last downloaded result must be the device step's result (same inputs)
-    e2e_same = bool(torch.equal(res_host[(n_e2e - 1) % 2].cuda(), out))
+    # the last downloaded result must be the device step's result (same inputs, same set)
+    run.step(i=n_e2e - 1)
+    torch.cuda.synchronize()
+    e2e_same = bool(torch.equal(res_host[(n_e2e - 1) % 2].cuda(), run.out))
+    del sets, outs
 
     flops = w.attn_flops()
     ms_step = elapsed_ms / K
@@ -545,14 +720,10 @@ def main():
     e2e_value = job_throughput(flops, world, e2e_ms)
 
     att_tflops = flops / (t_att * 1e-3) / 1e12
-    mod_bytes = 4.0 * rows * D
-    res_bytes = 6.0 * rows * D
-    mod_gbs = mod_bytes / (t_mod * 1e-3) / 1e9
-    res_gbs = res_bytes / (t_res * 1e-3) / 1e9
-    rope_bytes = 8.0 * rows * H * d  # q and k read, rotated q and k written, bf16
-    rope_gbs = rope_bytes / (t_rope * 1e-3) / 1e9 if args.rope_mode == "prepass" else None
     per_head = ATTN_DRAM_BYTES_PER_HEAD_480P.get(args.rope_mode) if w.name == "480p" else None
     traffic = per_head * H if per_head is not None and args.attn_variant == 0 else None
+    t["step_ms"] = elapsed_ms / K
+    head_fig = workload_figures(w, t, pk, args.rope_mode)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -560,52 +731,72 @@ def main():
         cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
                "seconds": dt}
         # the step's attention output on the same sampled rows, against the oracle
+        run.step(i=0)
         s_rows, ref_o = cpu_oracle_attention.last
         got = o[torch.from_numpy(s_rows).cuda()].float().cpu().double().numpy()
         err = np.abs(got - ref_o)
         cpu["parity"] = {"rows": int(len(s_rows)), "max_abs": float(err.max()),
                          "mean_abs": float(err.mean()), "tolerance_max_mean": [2e-2, 2e-3]}
+    del inp
+    run.free()
+    del run, dev, o, u, x_next, u_vel, q_rot, host
+    torch.cuda.empty_cache()
+
+    # the other workloads, each on its own seeded inputs, timed the same way (fewer steps)
+    workloads = {w.name: dict(head_fig, headline=True)}
+    if not args.no_workloads and not args.heads:
+        for name in wl.WORKLOADS:
+            if name == w.name:
+                continue
+            ww = wl.get_workload(name, args.seed)
+            r2 = StepRunner(ww, seed, args, torch, dit3d)
+            t2 = r2.timed(max(args.workload_steps, 1), args.warmup, barrier, local_rank)
+            t2["step_ms"] = t2["elapsed_ms"] / max(args.workload_steps, 1)
+            workloads[name] = workload_figures(ww, t2, pk, args.rope_mode)
+            workloads[name]["steps"] = max(args.workload_steps, 1)
+            r2.free()
+            del r2
 
     if rank == 0:
+        launches_per_step = 4 if args.rope_mode == "prepass" else 3
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded bf16 N(0,1) x/q/k/v, N(0,0.1) adaLN params)",
             "config": workload_config(w, world),
-            "gpu_launches": (4 if args.rope_mode == "prepass" else 3) * K,
+            "gpu_launches": launches_per_step * K,
             "roofline": {"bound": "tensor", "achieved": att_tflops,
-                         "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": att_tflops / pk["bf16_tflops_sustained"],
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": att_tflops / pk["bf16_tflops"],
+                         "frac_sustained": att_tflops / pk["bf16_tflops_sustained"],
                          "traffic": traffic,
                          "kernel": {"prepass": "dit_attn_fwd (operands rotated by dit_rope3d_qk)",
                                     "fused": "dit_attn_fwd (fused 3D-RoPE)",
                                     "none": "dit_attn_fwd without RoPE"}[args.rope_mode],
                          "attn_variant": ["single CTA", "CTA pair (cta_group::2)"][args.attn_variant],
-                         "peak_source": f"{pk['source']} sustained bf16 "
-                                        f"(burst {pk['bf16_tflops']}: frac "
-                                        f"{att_tflops / pk['bf16_tflops']:.3f})"},
+                         "peak_source": f"{pk['source']} burst bf16 {pk['bf16_tflops']} TFLOP/s "
+                                        f"(sustained {pk['bf16_tflops_sustained']}: frac_sustained)"},
             "components": {
-                "adaln_modulate": {"ms": t_mod, "GB/s": mod_gbs, "frac_hbm": mod_gbs / pk["hbm_gbs"],
-                                   "bytes": mod_bytes},
-                "rope3d_qk": ({"ms": t_rope, "GB/s": rope_gbs, "frac_hbm": rope_gbs / pk["hbm_gbs"],
-                               "bytes": rope_bytes} if args.rope_mode == "prepass" else None),
-                "attn_fwd": {"ms": t_att, "TFLOP/s": att_tflops, "flops": flops},
-                "gated_residual": {"ms": t_res, "GB/s": res_gbs, "frac_hbm": res_gbs / pk["hbm_gbs"],
-                                   "bytes": res_bytes},
-                "flow_euler_step": {"ms": t_euler, "GB/s": res_bytes / (t_euler * 1e-3) / 1e9,
-                                    "frac_hbm": res_bytes / (t_euler * 1e-3) / 1e9 / pk["hbm_gbs"],
-                                    "bytes": res_bytes, "in_step": False,
+                "adaln_modulate": head_fig["adaln_modulate"],
+                "rope3d_qk": head_fig["rope3d_qk"],
+                "attn_fwd": head_fig["attn_fwd"],
+                "gated_residual": head_fig["gated_residual"],
+                "flow_euler_step": {"ms": t_euler, "GB/s": 6.0 * rows * D / (t_euler * 1e-3) / 1e9,
+                                    "frac_hbm": 6.0 * rows * D / (t_euler * 1e-3) / 1e9 / pk["hbm_gbs"],
+                                    "bytes": 6.0 * rows * D, "in_step": False,
                                     "note": "sampler update x += dt_frame * u, timed separately"},
                 "attn_fwd_qk8": fp8,
                 **lin,
             },
+            "workloads": workloads,
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "pipelined": "2 buffer sets; uploads and downloads overlap neighbouring steps",
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                     "result_matches_device_step": e2e_same},
             "cpu_baseline": cpu,
+            "peaks": {k: pk[k] for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained", "source")},
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -74,7 +74,13 @@ struct Params {
   RopeParams rope;
   int32_t force_timeout;
   float o_scale;              // multiplies O in the epilogue (V's dequantisation scale; 1 else)
+  uint64_t wait_limit_ns;     // bound of the waits that give up the CTA's work (2 s by default)
+  // packed batches of up to kMaxOrder sequences: their order, longest first, on a 1-D
+  // grid (n_order > 0); otherwise a (pairs, heads) grid in cu_seqlens order
+  int32_t n_order;
+  int32_t seq_order[64];
 };
+constexpr int kMaxOrder = 64;
 
 template <int D>
 struct Smem {
@@ -101,6 +107,17 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^t of a pair of scores on the MUFU unit (ex2.approx). Moving a share of these to
+// an FMA-pipe polynomial (Cody-Waite reduction, degree-3 minimax) was measured slower
+// on B200 (a quarter of the pairs: -7 %; half: -15 %): the softmax warp's issue, not
+// the MUFU rate, sets its pace.
+__device__ __forceinline__ void exp2_pair(uint64_t t2, float& e0, float& e1) {
+  float t0, t1;
+  f2_unpack(t2, t0, t1);
+  e0 = ex2(t0);
+  e1 = ex2(t1);
 }
 
 // Byte offset of the 16-byte chunk `cc` (8 bf16) of row r inside a 128-row tile
@@ -243,12 +260,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int head = blockIdx.y;
+  int head = blockIdx.y;
 
-  // ---- work decode: which sequence and which pair of query tiles
+  // ---- work decode: which sequence, head and pair of query tiles
   int64_t seq_start, seq_len;
   int pair;
-  if (p.cu_seqlens == nullptr) {
+  if (p.n_order > 0) {
+    // packed batch, longest sequence first (1-D grid): every head of a sequence, then the
+    // next sequence, so the CTAs that finish last are those of the shortest sequences
+    int rem = blockIdx.x;
+    head = 0;
+    pair = 0;
+    seq_start = 0;
+    seq_len = 0;
+    for (int i = 0; i < p.n_order; ++i) {
+      const int s = p.seq_order[i];
+      const int64_t a = __ldg(p.cu_seqlens + s), b = __ldg(p.cu_seqlens + s + 1);
+      const int np = static_cast<int>((b - a + 2 * kTileM - 1) / (2 * kTileM));
+      if (rem < np * p.H) {
+        head = rem / np;
+        pair = rem - head * np;
+        seq_start = a;
+        seq_len = b - a;
+        break;
+      }
+      rem -= np * p.H;
+    }
+  } else if (p.cu_seqlens == nullptr) {
     const int seq = blockIdx.x / p.pairs_per_dense_seq;
     pair = blockIdx.x - seq * p.pairs_per_dense_seq;
     seq_len = p.dense_len;
@@ -330,7 +368,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       // warp-uniform decision: tcgen05.ld/st below are warp-collective
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_s, j & 1, abort))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_s, j & 1, abort, p.wait_limit_ns))) { ok = false; break; }
       ptx::tc_fence_after();
       uint32_t sr[128];
 #pragma unroll
@@ -383,9 +421,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const uint64_t t2 = f2_fma(f2_pack(s[32 * q4 + 2 * c], s[32 * q4 + 2 * c + 1]), sc2, nm2);
-          float t0, t1;
-          f2_unpack(t2, t0, t1);
-          const float e0 = ex2(t0), e1 = ex2(t1);
+          float e0, e1;
+          exp2_pair(t2, e0, e1);
           l2 = f2_add(l2, f2_pack(e0, e1));
           if constexpr (PV8) {
             const uint32_t h = e4m3x2(e0, e1);
@@ -408,7 +445,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ptx::mbar_arrive(bar_p);
     }
     // ---- epilogue: O / l -> bf16 -> global, plus the log-sum-exp
-    if (__all_sync(0xffffffffu, ok && ptx::mbar_wait(ptx::smem_u32(&b->o_final), 0, abort))) {
+    if (__all_sync(0xffffffffu, ok && ptx::mbar_wait(ptx::smem_u32(&b->o_final), 0, abort, p.wait_limit_ns))) {
       ptx::tc_fence_after();
       const int64_t row_in_seq = q_row0 + qi * kTileM + r;
       const bool valid = row_in_seq < seq_len;
@@ -465,7 +502,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int j = 0; j < nk; ++j) {
           const int st = j % stages;
           if (j >= stages &&
-              !ptx::mbar_wait(ptx::smem_u32(&empty[st]), ((j / stages) - 1) & 1, abort))
+              !ptx::mbar_wait(ptx::smem_u32(&empty[st]), ((j / stages) - 1) & 1, abort, p.wait_limit_ns))
             break;
           const int y = static_cast<int>(seq_start + static_cast<int64_t>(j) * kTileN);
           const uint32_t f = ptx::smem_u32(&full[st]);
@@ -539,17 +576,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
       // both halves, the second once the softmax has stored all of P
       auto pv_tile = [&](int qi, int st, bool acc, int j) -> bool {
-        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_half[qi]), j & 1, abort)) return false;
+        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_half[qi]), j & 1, abort, p.wait_limit_ns)) return false;
         ptx::tc_fence_after();
         pv(qi, st, acc, 0);
-        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_full[qi]), j & 1, abort)) return false;
+        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_full[qi]), j & 1, abort, p.wait_limit_ns)) return false;
         ptx::tc_fence_after();
         pv(qi, st, acc, 1);
         return true;
       };
       const uint32_t q_wait = ptx::smem_u32(p.use_rope ? &b->q_ready : &b->q_full);
-      bool ok = ptx::mbar_wait(q_wait, 0, abort);
-      if (ok) ok = ptx::mbar_wait(ptx::smem_u32(p.use_rope ? &b->k_ready[0] : &b->k_full[0]), 0, abort);
+      bool ok = ptx::mbar_wait(q_wait, 0, abort, p.wait_limit_ns);
+      if (ok) ok = ptx::mbar_wait(ptx::smem_u32(p.use_rope ? &b->k_ready[0] : &b->k_full[0]), 0, abort, p.wait_limit_ns);
       if (ok) {
         ptx::tc_fence_after();
         qk(0, 0);
@@ -561,11 +598,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int vs = j % kVStages, vph = (j / kVStages) & 1;
         const int ks1 = (j + 1) % kKStages, kph1 = ((j + 1) / kKStages) & 1;
         const bool more = j + 1 < nk;
-        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[vs]), vph, abort))) break;
+        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[vs]), vph, abort, p.wait_limit_ns))) break;
         if (!(ok = pv_tile(0, vs, j > 0, j))) break;
         if (more) {
           if (!(ok = ptx::mbar_wait(
-                    ptx::smem_u32(p.use_rope ? &b->k_ready[ks1] : &b->k_full[ks1]), kph1, abort)))
+                    ptx::smem_u32(p.use_rope ? &b->k_ready[ks1] : &b->k_full[ks1]), kph1, abort, p.wait_limit_ns)))
             break;
           ptx::tc_fence_after();
           qk(0, ks1);
@@ -604,7 +641,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tab_in_smem) rope_tile_smem<D>(ptx::smem_u32(tile), row0, nv, p.rope, tab, rt);
         else rope_tile_global<D>(tile, row0, nv, p.rope, rt);
       };
-      if (ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort)) {
+      if (ptx::mbar_wait(ptx::smem_u32(&b->q_full), 0, abort, p.wait_limit_ns)) {
         for (int qi = 0; qi < 2; ++qi) {
           const int64_t r0 = q_row0 + qi * kTileM;
           const int64_t rem = seq_len - r0;
@@ -615,7 +652,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
         for (int j = 0; j < nk; ++j) {
           const int st = j % kKStages, ph = (j / kKStages) & 1;
-          if (!ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort)) break;
+          if (!ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort, p.wait_limit_ns)) break;
           const int nv = (j == nk - 1) ? last_valid : kTileN;
           rope_tile(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv);
           ptx::fence_proxy_async_smem();

@@ -41,6 +41,7 @@ namespace dit3d {
 namespace attn2 {
 
 using attn::ex2;
+using attn::exp2_pair;
 using attn::lds128;
 using attn::lds128f;
 using attn::lds128_ordered;
@@ -320,9 +321,8 @@ attn_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const uint64_t t2 = f2_fma(f2_pack(s[32 * q4 + 2 * c], s[32 * q4 + 2 * c + 1]), sc2, nm2);
-          float t0, t1;
-          f2_unpack(t2, t0, t1);
-          const float e0 = ex2(t0), e1 = ex2(t1);
+          float e0, e1;
+          exp2_pair(t2, e0, e1);
           l2 = f2_add(l2, f2_pack(e0, e1));
           pw[c] = pack_bf16x2(e0, e1);
         }

@@ -1,11 +1,14 @@
 // C ABI of libdit3d (declared in include/dit3d.h): argument validation, tensor
 // maps, the RoPE cos/sin table cache and kernel launches. All device work is in
 // the kernels of adaln.cuh, rope3d.cuh and attn_fwd.cuh.
+#include <algorithm>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <thread>
 #include <tuple>
 #include <vector>
 
@@ -29,6 +32,7 @@ namespace {
 
 std::mutex g_mu;
 int g_force_timeout = 0;
+uint64_t g_wait_limit_ns = 2000000000ull;  // bound of the single-CTA kernels' waits
 int g_linear_variant = 0;  // 0: one CTA per 128x256 tile; 1: CTA pairs per 256x256 tile
 int g_attn_variant = 0;  // 0: one CTA per query-tile pair; 1: CTA pairs (head_dim 128)
 
@@ -134,36 +138,32 @@ void rope_table_layout(const dit_rope3d_desc* r, int t_ext, RopeParams* rp) {
   rp->n_entries = n;
 }
 
-// Host values of the table: cos/sin of the angle (pos + offset) * base^(-2i/d_a) in
-// fp64, stored fp32; a chunk's floats are (cos p0, cos p1, sin p0, sin p1, cos p2,
-// cos p3, sin p2, sin p3), pairs outside the band hold the identity.
-void rope_table_values(const dit_rope3d_desc* r, int t_ext, const RopeParams& rp,
-                       std::vector<float2>* out) {
+// What the fill kernel needs besides the layout: band widths, extents, offsets,
+// first pairs and the base.
+RopeTableSpec rope_table_spec(const dit_rope3d_desc* r, int t_ext, const RopeParams& rp) {
+  RopeTableSpec s{};
+  s.base = r->base;
   const int width[3] = {r->d_t, r->d_h, r->d_w};
   const int ext[3] = {t_ext, r->grid_h, r->grid_w};
   const int offs[3] = {r->t0, r->h0, r->w0};
   const int first_pair[3] = {0, r->d_t / 2, (r->d_t + r->d_h) / 2};
-  const int off[3] = {rp.off0, rp.off1, rp.off2}, str[3] = {rp.str0, rp.str1, rp.str2},
-            cf[3] = {rp.cf0, rp.cf1, rp.cf2};
-  out->assign(std::max(rp.n_entries, 2), make_float2(1.f, 0.f));  // (1,1,0,0) per couple
-  float* f = reinterpret_cast<float*>(out->data());
-  for (size_t i = 0; i < 2 * out->size(); ++i) f[i] = (i & 2) ? 0.f : 1.f;
   for (int a = 0; a < 3; ++a) {
-    const int np = width[a] / 2;
-    if (np == 0) continue;
-    for (int pos = 0; pos < ext[a]; ++pos)
-      for (int p = 4 * cf[a]; p < 4 * cf[a] + str[a] - 2; ++p) {
-        const int i = p - first_pair[a];
-        if (i < 0 || i >= np) continue;  // outside the band: identity
-        const double theta = std::pow(static_cast<double>(r->base), -2.0 * i / width[a]);
-        const double phi = static_cast<double>(pos + offs[a]) * theta;
-        const int e = p - 4 * cf[a];                        // pair index from the row start
-        float* chunk = f + 2 * (off[a] + pos * str[a]) + 8 * (e >> 2);
-        const int u = (e & 3) >> 1, w = e & 1;              // couple, pair within couple
-        chunk[4 * u + w] = static_cast<float>(std::cos(phi));
-        chunk[4 * u + 2 + w] = static_cast<float>(std::sin(phi));
-      }
+    s.width[a] = width[a];
+    s.ext[a] = ext[a];
+    s.offs[a] = offs[a];
+    s.first_pair[a] = first_pair[a];
   }
+  s.n_fill = std::max(rp.n_entries, 2);
+  return s;
+}
+
+// Writes the table of descriptor `r` into `dst` (at least max(n_entries, 2) float2) with
+// one kernel on `stream`: no host buffer, no copy.
+int fill_table(float2* dst, const dit_rope3d_desc* r, int t_ext, const RopeParams& rp,
+               cudaStream_t stream) {
+  const RopeTableSpec spec = rope_table_spec(r, t_ext, rp);
+  rope_table_fill_kernel<<<(spec.n_fill + 255) / 256, 256, 0, stream>>>(dst, rp, spec);
+  return launch_status();
 }
 
 // Cached device copy of the table for a descriptor (allocated once per device).
@@ -180,15 +180,15 @@ int get_table(const dit_rope3d_desc* r, int t_ext, cudaStream_t stream, RopePara
     rp->table = it->second;
     return DIT_OK;
   }
-  std::vector<float2> host;
-  rope_table_values(r, t_ext, *rp, &host);
   float2* dptr = nullptr;
-  if (cudaMalloc(&dptr, sizeof(float2) * host.size()) != cudaSuccess) return DIT_ERR_ALLOC;
-  // pageable source: the copy has consumed `host` when the call returns
-  if (cudaMemcpyAsync(dptr, host.data(), sizeof(float2) * host.size(), cudaMemcpyHostToDevice,
-                      stream) != cudaSuccess) {
+  if (cudaMalloc(&dptr, sizeof(float2) * std::max(rp->n_entries, 2)) != cudaSuccess)
+    return DIT_ERR_ALLOC;
+  // the table is shared by later calls on any stream: let its fill finish first
+  int s = fill_table(dptr, r, t_ext, *rp, stream);
+  if (s == DIT_OK && cudaStreamSynchronize(stream) != cudaSuccess) s = DIT_ERR_LAUNCH;
+  if (s != DIT_OK) {
     cudaFree(dptr);
-    return DIT_ERR_LAUNCH;
+    return s;
   }
   g_tables.emplace(key, dptr);
   rp->table = dptr;
@@ -236,6 +236,23 @@ bool make_tmap8(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Longest-first order of a packed batch for the single-CTA attention kernel (fills
+// prm->seq_order; stable for equal lengths). Left empty (natural order on a 2-D grid)
+// for dense batches, more than attn::kMaxOrder sequences, or a grid too large for 1-D.
+void set_seq_order(attn::Params* prm, const std::vector<int64_t>& lens, int64_t n_work, int32_t H,
+                   bool packed) {
+  prm->n_order = 0;
+  if (!packed || lens.size() > static_cast<size_t>(attn::kMaxOrder) ||
+      n_work * H >= (int64_t(1) << 31))
+    return;
+  std::vector<int32_t> order(lens.size());
+  for (size_t i = 0; i < order.size(); ++i) order[i] = static_cast<int32_t>(i);
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int32_t a, int32_t b) { return lens[a] > lens[b]; });
+  for (size_t i = 0; i < order.size(); ++i) prm->seq_order[i] = order[i];
+  prm->n_order = static_cast<int32_t>(order.size());
+}
+
 // F8: 0 all bf16; 1 E4M3 q and k; 2 E4M3 q, k and v (see attn_fwd_kernel)
 template <int D, int F8 = 0>
 int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32_t H,
@@ -257,7 +274,8 @@ int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32
       return DIT_ERR_LAUNCH;
     attr_set[dev] = true;
   }
-  dim3 grid(n_work, H);
+  // packed: 1-D grid over (sequence in prm.seq_order, head, pair); else (pairs, heads)
+  const dim3 grid = prm.n_order > 0 ? dim3(static_cast<unsigned>(n_work) * H) : dim3(n_work, H);
   attn::attn_fwd_kernel<D, F8><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
   return launch_status();
 }
@@ -267,6 +285,7 @@ int launch_attn_2sm(const void* q, const void* k, const void* v, int64_t rows, i
                     attn::Params prm, const std::vector<int64_t>& lens, bool dense,
                     cudaStream_t stream) {
   constexpr int D = attn2::kD;
+  prm.n_order = 0;  // the pair kernel walks packed sequences in cu_seqlens order
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, rows, static_cast<int64_t>(H) * D, 128) ||
       !make_tmap(&tk, k, rows, static_cast<int64_t>(H) * D, attn2::kHalfN) ||
@@ -297,10 +316,20 @@ int launch_attn_2sm(const void* q, const void* k, const void* v, int64_t rows, i
   return launch_status();
 }
 
+// Parameter groups shorter than this many rows (a group per frame) take the form that
+// loads gamma and beta with x (see adaln_modulate_kernel).
+constexpr int64_t kEarlyParamRows = 8192;
+
 template <int NV>
 void launch_modulate(const void* x, const void* g, const void* b, void* o, int64_t rows, int32_t D,
                      int64_t rpg, float eps, float s0, cudaStream_t st) {
-  adaln_modulate_kernel<NV><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+  if (rpg < kEarlyParamRows) {
+    adaln_modulate_kernel<NV, true><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
+        static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
+    return;
+  }
+  adaln_modulate_kernel<NV, false><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
       static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
 }
@@ -462,6 +491,7 @@ static int linear_impl(const void* x, const void* w, const void* bias, void* out
   prm.k_blocks = (K + k_per_stage - 1) / k_per_stage;
   prm.acc_scale = acc_scale;
   prm.force_timeout = g_force_timeout;
+  prm.wait_limit_ns = g_wait_limit_ns;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -500,6 +530,59 @@ static int linear_impl(const void* x, const void* w, const void* bias, void* out
   return launch_status();
 }
 
+
+// bf16 attention behind dit_attn_fwd and dit_attn_fwd_noalloc: argument checks, work
+// count, launch. `table` provides the RoPE cos/sin table (cached, or the fixed array).
+template <typename TableFn>
+int attn_bf16_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t rows,
+                   int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                   const int32_t* cu_seqlens_host, float softmax_scale,
+                   const dit_rope3d_desc* rope, void* stream, TableFn table) {
+  if (!q || !k || !v || !o) return DIT_ERR_NULL;
+  if (rows <= 0 || H <= 0 || H > 65535 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
+  if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;  // TMA row coordinates are int32
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return DIT_ERR_ALIGN;
+  std::vector<int64_t> lens;
+  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
+  int t_ext = 0;
+  if (rope)
+    if (int s = validate_rope(rope, d, lens, &t_ext)) return s;
+  if (int s = check_device()) return s;
+  auto st = static_cast<cudaStream_t>(stream);
+
+  attn::Params prm{};
+  prm.cu_seqlens = cu_seqlens_dev;
+  prm.n_seq = n_seq;
+  prm.H = H;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.force_timeout = g_force_timeout;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  prm.o_scale = 1.f;
+  int64_t n_work = 0;
+  if (cu_seqlens_dev == nullptr) {
+    prm.dense_len = rows / n_seq;
+    prm.pairs_per_dense_seq = static_cast<int32_t>((prm.dense_len + 2 * attn::kTileM - 1) / (2 * attn::kTileM));
+    n_work = static_cast<int64_t>(prm.pairs_per_dense_seq) * n_seq;
+  } else {
+    for (int64_t L : lens) n_work += (L + 2 * attn::kTileM - 1) / (2 * attn::kTileM);
+  }
+  if (n_work == 0) return DIT_OK;
+  if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
+  if (rope) {
+    prm.use_rope = 1;
+    if (int s = table(rope, t_ext, st, &prm.rope)) return s;
+  }
+  set_seq_order(&prm, lens, n_work, H, cu_seqlens_dev != nullptr);
+  if (d == 128 && g_attn_variant == 1)
+    return launch_attn_2sm(q, k, v, rows, H, prm, lens, cu_seqlens_dev == nullptr, st);
+  if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+  return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+}
 
 extern "C" {
 
@@ -559,48 +642,8 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
                  const int32_t* cu_seqlens_host, float softmax_scale, const dit_rope3d_desc* rope,
                  void* stream) {
-  if (!q || !k || !v || !o) return DIT_ERR_NULL;
-  if (rows <= 0 || H <= 0 || H > 65535 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
-  if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;  // TMA row coordinates are int32
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-    return DIT_ERR_ALIGN;
-  std::vector<int64_t> lens;
-  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
-  int t_ext = 0;
-  if (rope)
-    if (int s = validate_rope(rope, d, lens, &t_ext)) return s;
-  if (int s = check_device()) return s;
-  auto st = static_cast<cudaStream_t>(stream);
-
-  attn::Params prm{};
-  prm.cu_seqlens = cu_seqlens_dev;
-  prm.n_seq = n_seq;
-  prm.H = H;
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.lse = lse;
-  prm.force_timeout = g_force_timeout;
-  prm.o_scale = 1.f;
-  int64_t n_work = 0;
-  if (cu_seqlens_dev == nullptr) {
-    prm.dense_len = rows / n_seq;
-    prm.pairs_per_dense_seq = static_cast<int32_t>((prm.dense_len + 2 * attn::kTileM - 1) / (2 * attn::kTileM));
-    n_work = static_cast<int64_t>(prm.pairs_per_dense_seq) * n_seq;
-  } else {
-    for (int64_t L : lens) n_work += (L + 2 * attn::kTileM - 1) / (2 * attn::kTileM);
-  }
-  if (n_work == 0) return DIT_OK;
-  if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
-  if (rope) {
-    prm.use_rope = 1;
-    if (int s = get_table(rope, t_ext, st, &prm.rope)) return s;
-  }
-  if (d == 128 && g_attn_variant == 1)
-    return launch_attn_2sm(q, k, v, rows, H, prm, lens, cu_seqlens_dev == nullptr, st);
-  if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
-  return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+  return attn_bf16_impl(q, k, v, o, lse, rows, H, d, n_seq, cu_seqlens_dev, cu_seqlens_host,
+                        softmax_scale, rope, stream, get_table);
 }
 
 }  // extern "C"
@@ -631,6 +674,7 @@ int attn_fp8_impl(const void* q8, const void* k8, const void* v, void* o, float*
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.force_timeout = g_force_timeout;
+  prm.wait_limit_ns = g_wait_limit_ns;
   prm.o_scale = v8 ? v_scale : 1.f;
   int64_t n_work = 0;
   if (cu_seqlens_dev == nullptr) {
@@ -643,6 +687,7 @@ int attn_fp8_impl(const void* q8, const void* k8, const void* v, void* o, float*
   }
   if (n_work == 0) return DIT_OK;
   if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
+  set_seq_order(&prm, lens, n_work, H, cu_seqlens_dev != nullptr);
   return v8 ? launch_attn<128, 2>(q8, k8, v, rows, H, prm, static_cast<int>(n_work), st)
             : launch_attn<128, 1>(q8, k8, v, rows, H, prm, static_cast<int>(n_work), st);
 }
@@ -683,6 +728,75 @@ int dit_quantize_e4m3(const void* x, void* out8, int64_t n, float inv_scale, voi
   return launch_status();
 }
 
+}  // extern "C"
+
+namespace {
+// Host watchdog loop: polls ready() (1 done, 0 not yet, -1 failed) until it is done or
+// fails, or until timeout_us of wall time have passed since the first poll; sleeps
+// between polls, from 1 us doubling up to 100 us.
+template <typename Ready>
+int poll_until(Ready ready, int64_t timeout_us) {
+  const auto t0 = std::chrono::steady_clock::now();
+  int64_t nap = 1;
+  for (;;) {
+    const int r = ready();
+    if (r > 0) return DIT_OK;
+    if (r < 0) return DIT_ERR_LAUNCH;
+    const int64_t waited = std::chrono::duration_cast<std::chrono::microseconds>(
+                               std::chrono::steady_clock::now() - t0).count();
+    if (waited >= timeout_us) return DIT_ERR_TIMEOUT;
+    std::this_thread::sleep_for(std::chrono::microseconds(std::min(nap, timeout_us - waited)));
+    nap = std::min<int64_t>(2 * nap, 100);
+  }
+}
+}  // namespace
+
+extern "C" {
+
+int dit_wait_device(void* stream, int64_t timeout_us) {
+  if (timeout_us < 0) return DIT_ERR_SHAPE;
+  auto st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return DIT_ERR_LAUNCH;
+  if (cudaEventRecord(ev, st) != cudaSuccess) {
+    cudaEventDestroy(ev);
+    return DIT_ERR_LAUNCH;
+  }
+  const int s = poll_until(
+      [&] {
+        const cudaError_t e = cudaEventQuery(ev);
+        return e == cudaSuccess ? 1 : (e == cudaErrorNotReady ? 0 : -1);
+      },
+      timeout_us);
+  cudaEventDestroy(ev);  // released once the recorded work completes
+  if (s != DIT_OK) return s;
+  // the stream has finished: read and clear the error word on it (no device-wide wait)
+  uint32_t err = 0;
+  const uint32_t zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&err, g_device_error, sizeof(err), 0, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return DIT_ERR_LAUNCH;
+  if (err != 0 && (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(zero), 0,
+                                           cudaMemcpyHostToDevice, st) != cudaSuccess ||
+                   cudaStreamSynchronize(st) != cudaSuccess))
+    return DIT_ERR_LAUNCH;
+  return (err & kDevErrTimeout) ? DIT_ERR_TIMEOUT : DIT_OK;
+}
+
+int dit_debug_poll_fake(int64_t busy_polls, int fail, int64_t timeout_us, int64_t* polls) {
+  int64_t n = 0;
+  const int s = poll_until(
+      [&] {
+        ++n;
+        if (n > busy_polls) return fail ? -1 : 1;
+        return 0;
+      },
+      timeout_us);
+  if (polls) *polls = n;
+  return s;
+}
+
 int dit_check_device(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DIT_ERR_LAUNCH;
   uint32_t err = 0, zero = 0;
@@ -692,19 +806,9 @@ int dit_check_device(void* stream) {
   return (err & kDevErrTimeout) ? DIT_ERR_TIMEOUT : DIT_OK;
 }
 
-void dit_shutdown(void) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  int cur = 0;
-  cudaGetDevice(&cur);
-  for (auto& kv : g_tables) {
-    cudaSetDevice(kv.first.dev);
-    cudaFree(kv.second);
-  }
-  g_tables.clear();
-  cudaSetDevice(cur);
-}
-
 void dit_debug_force_timeout(int enable) { g_force_timeout = enable ? 1 : 0; }
+
+void dit_debug_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 2000000000ull; }
 
 int dit_set_attn_variant(int variant) {
   if (variant != 0 && variant != 1) return DIT_ERR_SHAPE;
@@ -718,7 +822,7 @@ int dit_set_attn_variant(int variant) {
 // dit_attn_fwd_noalloc: the same attention, but the 3D-RoPE cos/sin table lives in a
 // fixed array of device memory that is part of the loaded library, so the call never
 // allocates. The array is shared by every call on a device and holds the last call's
-// table; the host rewrites the whole used range on every call.
+// table; every call rewrites the whole range it uses, with a kernel on its stream.
 namespace {
 
 constexpr int kNoAllocTableEntries = 65536;  // float2 entries: 512 KiB per device
@@ -736,8 +840,12 @@ int noalloc_table_address(float2** out) {
   auto it = g_noalloc_addr.find(dev);
   if (it == g_noalloc_addr.end()) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_rope_table) != cudaSuccess || ptr == nullptr)
-      return DIT_ERR_LAUNCH;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_rope_table);
+    if (e == cudaErrorMemoryAllocation) {
+      cudaGetLastError();  // not sticky: clear it
+      return DIT_ERR_ALLOC;  // loading the library's module onto the device needs memory
+    }
+    if (e != cudaSuccess || ptr == nullptr) return DIT_ERR_LAUNCH;
     it = g_noalloc_addr.emplace(dev, static_cast<float2*>(ptr)).first;
   }
   *out = it->second;
@@ -751,57 +859,34 @@ extern "C" int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int32_t n_seq, const int32_t* cu_seqlens_dev,
                                     const int32_t* cu_seqlens_host, float softmax_scale,
                                     const dit_rope3d_desc* rope, void* stream) {
-  if (!q || !k || !v || !o) return DIT_ERR_NULL;
-  if (rows <= 0 || H <= 0 || H > 65535 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
-  if (rows >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-    return DIT_ERR_ALIGN;
-  std::vector<int64_t> lens;
-  if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
-  int t_ext = 0;
-  if (rope)
-    if (int s = validate_rope(rope, d, lens, &t_ext)) return s;
-  if (int s = check_device()) return s;
-  auto st = static_cast<cudaStream_t>(stream);
-
-  attn::Params prm{};
-  prm.cu_seqlens = cu_seqlens_dev;
-  prm.n_seq = n_seq;
-  prm.H = H;
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.lse = lse;
-  prm.force_timeout = g_force_timeout;
-  prm.o_scale = 1.f;
-  int64_t n_work = 0;
-  if (cu_seqlens_dev == nullptr) {
-    prm.dense_len = rows / n_seq;
-    prm.pairs_per_dense_seq =
-        static_cast<int32_t>((prm.dense_len + 2 * attn::kTileM - 1) / (2 * attn::kTileM));
-    n_work = static_cast<int64_t>(prm.pairs_per_dense_seq) * n_seq;
-  } else {
-    for (int64_t L : lens) n_work += (L + 2 * attn::kTileM - 1) / (2 * attn::kTileM);
-  }
-  if (n_work == 0) return DIT_OK;
-  if (n_work > INT32_MAX) return DIT_ERR_SHAPE;
-  if (rope) {
-    std::vector<float2> host;
-    rope_table_layout(rope, t_ext, &prm.rope);
-    rope_table_values(rope, t_ext, prm.rope, &host);
-    if (prm.rope.n_entries > kNoAllocTableEntries) return DIT_ERR_SCRATCH;
+  // the table is written into the fixed array by a kernel on `stream`, ahead of the
+  // attention on the same stream
+  auto fixed_table = [](const dit_rope3d_desc* r, int t_ext, cudaStream_t st, RopeParams* rp) {
+    rope_table_layout(r, t_ext, rp);
+    if (std::max(rp->n_entries, 2) > kNoAllocTableEntries) return static_cast<int>(DIT_ERR_SCRATCH);
     float2* table = nullptr;
     if (int s = noalloc_table_address(&table)) return s;
-    // pageable source: the copy has consumed `host` when the call returns
-    if (cudaMemcpyAsync(table, host.data(), sizeof(float2) * host.size(), cudaMemcpyHostToDevice,
-                        st) != cudaSuccess)
-      return DIT_ERR_LAUNCH;
-    prm.use_rope = 1;
-    prm.rope.table = table;
+    rp->table = table;
+    return fill_table(table, r, t_ext, *rp, st);
+  };
+  return attn_bf16_impl(q, k, v, o, lse, rows, H, d, n_seq, cu_seqlens_dev, cu_seqlens_host,
+                        softmax_scale, rope, stream, fixed_table);
+}
+
+extern "C" void dit_shutdown(void) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto& kv : g_tables) {
+      cudaSetDevice(kv.first.dev);
+      cudaFree(kv.second);
+    }
+    g_tables.clear();
+    cudaSetDevice(cur);
   }
-  if (d == 128 && g_attn_variant == 1)
-    return launch_attn_2sm(q, k, v, rows, H, prm, lens, cu_seqlens_dev == nullptr, st);
-  if (d == 128) return launch_attn<128>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
-  return launch_attn<64>(q, k, v, rows, H, prm, static_cast<int>(n_work), st);
+  // the fixed array's addresses are looked up again on next use (a device reset
+  // between two uses would leave them stale)
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  g_noalloc_addr.clear();
 }

@@ -51,6 +51,7 @@ struct Params {
   int32_t tiles_m, tiles_n, k_blocks;
   int32_t force_timeout;
   float acc_scale;             // multiplies the accumulator (x_scale * w_scale for E4M3; 1 else)
+  uint64_t wait_limit_ns;      // bound of the waits that give up the CTA's work (2 s by default)
 };
 
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& tm, int& tn) {
@@ -167,7 +168,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % kStages;
           if (it >= kStages &&
-              !ptx::mbar_wait(ptx::smem_u32(&empty[s]), ((it / kStages) - 1) & 1, abort)) {
+              !ptx::mbar_wait(ptx::smem_u32(&empty[s]), ((it / kStages) - 1) & 1, abort, p.wait_limit_ns)) {
             ok = false;
             break;
           }
@@ -194,14 +195,14 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
         const int b = local & 1;
         const uint32_t acc = tmem + static_cast<uint32_t>(b * kBN);
         if (local >= 2 &&
-            !ptx::mbar_wait(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1, abort)) {
+            !ptx::mbar_wait(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1, abort, p.wait_limit_ns)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % kStages;
-          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages) & 1, abort)) {
+          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages) & 1, abort, p.wait_limit_ns)) {
             ok = false;
             break;
           }
@@ -239,7 +240,7 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
     int local = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++local) {
       const int b = local & 1;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&acc_full[b]), (local / 2) & 1, abort)))
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&acc_full[b]), (local / 2) & 1, abort, p.wait_limit_ns)))
         break;
       ptx::tc_fence_after();
       int tm, tn;

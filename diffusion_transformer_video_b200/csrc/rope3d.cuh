@@ -8,7 +8,7 @@
 // pos * base^(-2i/d_a), rotation [[cos, -sin], [sin, cos]], positions counted from
 // 0 at each sequence start plus a constant offset.
 //
-// cos/sin come from a table the host fills in fp64 and stores in fp32, laid out so
+// cos/sin come from a table computed in fp64 and stored in fp32, laid out so
 // that one 16-byte data chunk (8 bf16 = 4 pairs) needs two 16-byte table reads.
 // For band a (t, h, w) the table holds, per position pos, the values of every pair
 // of the chunks the band touches -- chunk-aligned, pairs outside the band set to the
@@ -95,6 +95,49 @@ __device__ __forceinline__ uint4 rope_chunk(const RopeParams& rp, const float2* 
   }
   return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                     pack_bf16x2(x[6], x[7]));
+}
+
+// What the table holds, per band a (t, h, w): its width d_a, its number of positions,
+// its position offset and the head pair where it starts; the frequency base.
+struct RopeTableSpec {
+  float base;
+  int32_t width[3], ext[3], offs[3], first_pair[3];
+  int32_t n_fill;  // float2 entries to write (n_entries, at least 2)
+};
+
+// Writes the cos/sin table of the layout above, one float2 entry per thread: for pair
+// i of band a at position pos, the angle (pos + offset_a) * base^(-2i/d_a) in fp64,
+// its cosine and sine rounded to fp32. Entries outside every band, pairs of a chunk
+// outside its band, and the two padding entries that end each position's row hold the
+// identity (cos 1, sin 0): even entries are cosine couples, odd ones sine couples.
+__global__ void __launch_bounds__(256)
+rope_table_fill_kernel(float2* __restrict__ table, RopeParams rp, RopeTableSpec s) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= s.n_fill) return;
+  const int off[3] = {rp.off0, rp.off1, rp.off2};
+  const int str[3] = {rp.str0, rp.str1, rp.str2};
+  const int cf[3] = {rp.cf0, rp.cf1, rp.cf2};
+  const bool is_sin = (e & 1) != 0;
+  float res[2] = {is_sin ? 0.f : 1.f, is_sin ? 0.f : 1.f};
+  for (int a = 0; a < 3; ++a) {
+    if (str[a] == 0) continue;  // empty band: no section
+    const int r = e - off[a];
+    if (r < 0 || r >= s.ext[a] * str[a]) continue;
+    const int pos = r / str[a], k = r - pos * str[a];
+    if (k < str[a] - 2) {
+      const int u = (k & 3) >> 1;  // couple inside the chunk
+      for (int w = 0; w < 2; ++w) {
+        const int p = 4 * (cf[a] + (k >> 2)) + 2 * u + w;  // pair index in the head
+        const int i = p - s.first_pair[a];
+        if (i < 0 || 2 * i >= s.width[a]) continue;
+        const double theta = pow(static_cast<double>(s.base), -2.0 * i / s.width[a]);
+        const double phi = static_cast<double>(pos + s.offs[a]) * theta;
+        res[w] = static_cast<float>(is_sin ? sin(phi) : cos(phi));
+      }
+    }
+    break;
+  }
+  table[e] = make_float2(res[0], res[1]);
 }
 
 // Sequence start of global row `row` (largest s with cu[s] <= row).

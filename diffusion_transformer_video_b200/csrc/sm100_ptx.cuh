@@ -62,13 +62,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait on phase `parity` of an mbarrier. Gives up after `limit_ns`
-// of wall time, or as soon as another role of the CTA raised `*abort`.
+// of wall time, or as soon as another role of the CTA raised `*abort`; both are
+// checked after the first unsuccessful try and then every 256 tries.
 // Returns false when it gave up; the caller must then leave its loop.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort) return false;

@@ -26,7 +26,8 @@ EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "d
            "dit_set_linear_variant", "dit_attn_fwd_qk8", "dit_attn_fwd_fp8", "dit_quantize_e4m3",
            "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
-           "dit_set_attn_variant", "dit_debug_force_timeout")
+           "dit_set_attn_variant", "dit_debug_force_timeout",
+           "dit_debug_wait_limit_ns", "dit_wait_device", "dit_debug_poll_fake")
 
 
 class DitError(RuntimeError):
@@ -84,6 +85,12 @@ def lib():
         L.dit_set_attn_variant.restype = ctypes.c_int
         L.dit_debug_force_timeout.argtypes = [ctypes.c_int]
         L.dit_debug_force_timeout.restype = None
+        L.dit_debug_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.dit_debug_wait_limit_ns.restype = None
+        L.dit_wait_device.argtypes = [P, i64]
+        L.dit_wait_device.restype = ctypes.c_int
+        L.dit_debug_poll_fake.argtypes = [i64, ctypes.c_int, i64, ctypes.POINTER(i64)]
+        L.dit_debug_poll_fake.restype = ctypes.c_int
         for name in ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
                      "dit_check_device"):
             getattr(L, name).restype = ctypes.c_int
@@ -327,6 +334,13 @@ def dit_set_linear_variant(variant: int):
 def dit_check_device():
     """Synchronises the current stream and raises DitError if a kernel gave up a wait."""
     _check(lib().dit_check_device(_stream()))
+
+
+def dit_wait_device(timeout_us: int):
+    """Waits for the current stream for at most timeout_us of wall time (polling, no
+    blocking synchronisation); raises DitError with DIT_ERR_TIMEOUT if it has not
+    finished by then or if a kernel gave up a wait."""
+    _check(lib().dit_wait_device(_stream(), int(timeout_us)))
 
 
 def dit_shutdown():

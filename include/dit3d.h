@@ -25,9 +25,10 @@
  *    exceptions are stated at their calls (fp32 lse and dt: 4 bytes; the codes
  *    written by dit_quantize_e4m3: 8 bytes).
  *  - The caller owns every buffer. Calls allocate nothing per call; the RoPE
- *    cos/sin tables (fp64 on the host, stored fp32) are cached in device memory
- *    per (device, descriptor, extent) on first use and freed by dit_shutdown().
- *    Make the first call for a given RoPE descriptor outside CUDA-graph capture.
+ *    cos/sin tables (angles in fp64, stored fp32, written by a kernel) are cached in
+ *    device memory per (device, descriptor, extent) on first use and freed by
+ *    dit_shutdown(). The first call for a given RoPE descriptor allocates and waits for
+ *    its table: make it outside CUDA-graph capture.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only enqueue
  *    work: they return before the GPU has run it. Validation reads host data only.
  *  - Return value: DIT_OK or a dit_status code; nothing is printed, thrown or
@@ -187,8 +188,8 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 /* Allocation-free variant of dit_attn_fwd (no counterpart in the source pages).
  * Same arguments, layouts, results and errors as dit_attn_fwd; the difference is
  * where the 3D-RoPE cos/sin table lives. dit_attn_fwd allocates it with cudaMalloc
- * on first use and caches it; this call instead writes it (host-computed, the same
- * values) into a fixed array of device memory that belongs to the loaded library,
+ * on first use and caches it; this call instead writes it (the same values, by the
+ * same kernel) into a fixed array of device memory that belongs to the loaded library,
  * so it never calls cudaMalloc, cudaFree or any allocating routine. It is meant for
  * callers that must not allocate device memory while they run: processes that hand
  * all device memory to their own pool or allocator up front, memory-capped serving
@@ -196,13 +197,19 @@ int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  * device synchronisation.
  *   - The array holds at most 65536 (cos, sin) pairs (512 KiB); a larger table (long
  *     videos or large patch grids) returns DIT_ERR_SCRATCH and launches nothing.
- *   - Every GPU that loads the library holds the array until the process exits.
+ *   - Every GPU that loads the library holds the array until the process exits. The
+ *     driver places it when the library's device code is first loaded on a device,
+ *     which is the first libdit3d call there (lazy loading): make any one libdit3d
+ *     call on each device before handing the rest of its memory to a pool. If that
+ *     load finds no memory, this call returns DIT_ERR_ALLOC.
  *   - The first call on a device looks up the array's device address (a runtime
  *     query, no allocation); make that first call before any stream capture.
+ *     dit_shutdown() forgets the looked-up addresses.
  *   - All calls on a device share the one array, which keeps the last call's table:
- *     each call rewrites the whole range it uses (a copy on `stream` before the
- *     kernel), so calls whose work overlaps on the GPU (different streams without
- *     ordering) race on the array and must be serialised by the caller.
+ *     each call rewrites the whole range it uses (a fill kernel on `stream` before the
+ *     attention), so calls on one stream are ordered, but calls whose work overlaps on
+ *     the GPU (different streams without ordering) race on the array and must be
+ *     serialised by the caller.
  *   - With rope == NULL no table is involved and the call is dit_attn_fwd exactly. */
 int dit_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                          int64_t rows, int32_t H, int32_t d, int32_t n_seq,
@@ -223,12 +230,6 @@ int dit_attn_fwd_qk8(const void* q8, const void* k8, const void* v, void* o, flo
                      const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                      float softmax_scale, float q_scale, float k_scale, void* stream);
 
-/* out8[i] = e4m3(x[i] * inv_scale): FP8 E4M3 codes of bf16 values, rounded to nearest
- * even and saturated at +-448 (same page and section). x: n bf16 (16-byte aligned),
- * out8: n bytes (8-byte aligned), n % 8 == 0. With inv_scale a power of two the
- * product is exact, so every code is the nearest E4M3 value of x * inv_scale.
- * Errors: DIT_ERR_NULL, DIT_ERR_SHAPE (n < 0, n % 8, inv_scale not finite),
- * DIT_ERR_ALIGN. n == 0 is a no-op. */
 /* Attention with E4M3 q, k and v (same page and section): S = q_scale k_scale (q8 . k8)
  * and O = v_scale (P8 . v8) / l both run as kind::f8f6f4 MMAs, with P rounded to E4M3
  * (P <= 2^8 by the lazy running maximum, inside E4M3's range) and the row sum l
@@ -240,12 +241,34 @@ int dit_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* o, fl
                      float softmax_scale, float q_scale, float k_scale, float v_scale,
                      void* stream);
 
+/* out8[i] = e4m3(x[i] * inv_scale): FP8 E4M3 codes of bf16 values, rounded to nearest
+ * even and saturated at +-448 (same page and section). x: n bf16 (16-byte aligned),
+ * out8: n bytes (8-byte aligned), n % 8 == 0. With inv_scale a power of two the
+ * product is exact, so every code is the nearest E4M3 value of x * inv_scale.
+ * Errors: DIT_ERR_NULL, DIT_ERR_SHAPE (n < 0, n % 8, inv_scale not finite),
+ * DIT_ERR_ALIGN. n == 0 is a no-op. */
 int dit_quantize_e4m3(const void* x, void* out8, int64_t n, float inv_scale, void* stream);
 
 /* Waits for `stream`, then reads and clears the library's device error word.
  * Returns DIT_ERR_TIMEOUT if any kernel gave up a bounded wait since the last
  * check (its outputs are then invalid), DIT_ERR_LAUNCH on a CUDA error, else DIT_OK. */
 int dit_check_device(void* stream);
+
+/* Host watchdog form of dit_check_device: polls an event recorded on `stream` (no
+ * blocking synchronisation) for at most timeout_us microseconds of wall time. Returns
+ * DIT_ERR_TIMEOUT when the stream's work has not finished by then (the work keeps
+ * running and the call may be repeated; this is how a host learns of a kernel that
+ * stopped making progress without blocking on it), DIT_ERR_LAUNCH on a CUDA error;
+ * once the stream has finished, reads and clears the device error word on that stream
+ * and returns as dit_check_device does. DIT_ERR_SHAPE for a negative timeout. */
+int dit_wait_device(void* stream, int64_t timeout_us);
+
+/* Test hook of dit_wait_device's polling loop, with a fake query in place of the
+ * event: the query reports "not yet" busy_polls times, then "done" (fail == 0) or
+ * "failed" (fail != 0). Returns what dit_wait_device's loop returns (DIT_OK,
+ * DIT_ERR_LAUNCH, DIT_ERR_TIMEOUT) and stores the number of polls made in *polls
+ * (may be NULL). Needs no GPU. */
+int dit_debug_poll_fake(int64_t busy_polls, int fail, int64_t timeout_us, int64_t* polls);
 
 /* Human-readable name of a dit_status code (static string, never NULL). */
 const char* dit_status_string(int status);
@@ -266,6 +289,14 @@ int dit_set_attn_variant(int variant);
 /* Test hook: 1 makes the next attention launches give up their first wait at once
  * (exercising the bounded-wait error path without any hang), 0 restores. */
 void dit_debug_force_timeout(int enable);
+
+/* Test hook: the time limit, in nanoseconds, of the waits in later launches of the
+ * single-CTA attention and linear kernels (0 restores the default of 2 s). A limit of
+ * a few nanoseconds makes a wait that is not already satisfied run out: the kernel
+ * leaves its work, drains its copies and MMAs and raises the error that the next
+ * dit_check_device() returns as DIT_ERR_TIMEOUT. The CTA-pair kernels keep 2 s. A plain
+ * process-wide setting, not synchronised. */
+void dit_debug_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -86,3 +86,19 @@ def test_valid_call_without_gpu_reports_device_error(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.dit_adaln_modulate(FAKE, FAKE, FAKE, FAKE, 4, 64, 4, 1e-6, 1.0, None) == 5
+
+
+def test_watchdog_poll_loop_with_a_fake_query(L):
+    # dit_wait_device's polling loop, driven by a fake query instead of a CUDA event:
+    # done after 3 "not yet" answers, failed after 2, never done within 20 ms
+    import time
+    n = ctypes.c_int64(0)
+    assert L.dit_debug_poll_fake(3, 0, 1_000_000, ctypes.byref(n)) == 0 and n.value == 4
+    assert L.dit_debug_poll_fake(2, 1, 1_000_000, ctypes.byref(n)) == 6 and n.value == 3
+    t0 = time.perf_counter()
+    assert L.dit_debug_poll_fake(1 << 60, 0, 20_000, ctypes.byref(n)) == 7
+    waited = time.perf_counter() - t0
+    assert 0.02 <= waited < 2.0 and n.value > 2
+    assert L.dit_debug_poll_fake(0, 0, 0, None) == 0        # done at the first poll
+    assert L.dit_debug_poll_fake(5, 0, 0, None) == 7        # no time allowed
+    assert L.dit_wait_device(None, -1) == 2                 # rejected before any CUDA call

@@ -81,3 +81,40 @@ def test_guards_survive_every_kernel():
 
     bad = [name for name, ok in checks if not ok]
     assert not bad, f"guard regions overwritten by: {bad}"
+
+
+def _raw_attn(entry, q, k, v, o, lse, desc):
+    import ctypes
+    rows, H, d = q.shape
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    status = getattr(dit3d.lib(), entry)(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+        ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()), rows, H, d, 1, None, None,
+        0.0, None if desc is None else ctypes.byref(desc), st)
+    assert status == 0, dit3d.lib().dit_status_string(status)
+    dit3d.dit_check_device()
+
+
+@pytest.mark.parametrize("variant", [0, 1])
+def test_guards_survive_rope_attention_and_the_pair_kernel(variant):
+    # The CTA-pair kernel covers 512 query rows per pair, so 333 rows leave most of its
+    # last pair past the end; the in-kernel RoPE rotates the ragged tile in place; the
+    # allocation-free call writes its table into the library's own array.
+    g = torch.Generator(device="cuda").manual_seed(5)
+    rows, H, d = 333, 3, 128
+    bf = lambda *s: torch.randn(*s, device="cuda", generator=g).to(torch.bfloat16)
+    q, k, v = bf(rows, H, d), bf(rows, H, d), bf(rows, H, d)
+    desc = dit3d.rope_desc(9, 37, (44, 42, 42))
+    dit3d.dit_set_attn_variant(variant)
+    try:
+        bad = []
+        for entry, rope in (("dit_attn_fwd", None), ("dit_attn_fwd", desc),
+                            ("dit_attn_fwd_noalloc", desc)):
+            ob, o = _guarded((rows, H, d), torch.bfloat16)
+            lb, lse = _guarded((rows, H), torch.float32)
+            _raw_attn(entry, q, k, v, o, lse, rope)
+            if not (_intact(ob, o.numel()) and _intact(lb, lse.numel())):
+                bad.append((entry, rope is not None))
+        assert not bad, f"variant {variant}: guard regions overwritten by {bad}"
+    finally:
+        dit3d.dit_set_attn_variant(0)

@@ -30,6 +30,20 @@ def test_adaln_modulate_parity(rows, D, rpg, s0):
     check_modulation(from_dev(out), ref, f"modulate rows={rows} D={D}")
 
 
+@pytest.mark.parametrize("rows,D,rpg", [(9000, 3072, 1500), (4000, 5120, 400), (30000, 128, 1000),
+                                        (20000, 1032, 20)])
+def test_adaln_modulate_large_and_in_place(rows, D, rpg):
+    # many rows and groups (ragged widths included), out of place and in place over x
+    x, g, b = bits((rows, D)), bits((rows // rpg, D), 0.1), bits((rows // rpg, D), 0.1)
+    xt = to_dev(x)
+    out = dit3d.dit_adaln_modulate(xt, to_dev(g), to_dev(b), rpg)
+    ref = oracle.adaln_modulate(f64(x), f64(g), f64(b), rpg)
+    check_modulation(from_dev(out), ref, f"modulate rows={rows} D={D}")
+    dit3d.dit_adaln_modulate(xt, to_dev(g), to_dev(b), rpg, out=xt)
+    dit3d.dit_check_device()
+    assert torch.equal(xt, out)
+
+
 def test_adaln_modulate_in_place_and_constant_rows():
     rows, D = 6, 256
     x = np.repeat(wl.f32_to_bf16_bits(np.linspace(-3, 3, rows, dtype=np.float32))[:, None], D, 1)
@@ -278,3 +292,48 @@ def test_bounded_wait_reports_timeout_without_hanging():
     o = dit3d.dit_attn_fwd(q, q, q)
     dit3d.dit_check_device()
     assert torch.isfinite(o.float()).all()
+
+
+def test_a_wait_that_runs_out_reports_timeout():
+    # A wait limit of 1 ns: the first wait of the attention kernel that is not already
+    # satisfied runs out on its %globaltimer check (not the forced-abort path); the CTA
+    # leaves its work mid-pipeline, drains its copies and MMAs, frees tensor memory and
+    # raises the error bit, and the context stays usable.
+    g = torch.Generator(device="cuda").manual_seed(8)
+    q, k, v = [torch.randn(8192, 4, 128, device="cuda", generator=g).to(torch.bfloat16)
+               for _ in range(3)]
+    ref = dit3d.dit_attn_fwd(q, k, v)
+    dit3d.dit_check_device()
+    dit3d.lib().dit_debug_wait_limit_ns(1)
+    try:
+        dit3d.dit_attn_fwd(q, k, v)
+        with pytest.raises(dit3d.DitError) as e:
+            dit3d.dit_check_device()
+        assert e.value.status == 7
+    finally:
+        dit3d.lib().dit_debug_wait_limit_ns(0)
+    o = dit3d.dit_attn_fwd(q, k, v)
+    dit3d.dit_check_device()
+    assert torch.equal(o, ref)
+
+
+def test_host_watchdog_returns_while_work_runs_then_reports_success():
+    # dit_wait_device polls an event: on an attention that needs milliseconds, a 50 us
+    # limit returns DIT_ERR_TIMEOUT without blocking; a generous one then returns OK.
+    q = torch.randn(32768, 8, 128, device="cuda").to(torch.bfloat16)
+    dit3d.dit_check_device()
+    dit3d.dit_attn_fwd(q, q, q)
+    with pytest.raises(dit3d.DitError) as e:
+        dit3d.dit_wait_device(50)
+    assert e.value.status == 7
+    dit3d.dit_wait_device(60_000_000)
+    # and it reports a kernel that gave up a wait, as dit_check_device does
+    dit3d.lib().dit_debug_force_timeout(1)
+    try:
+        dit3d.dit_attn_fwd(q[:300], q[:300], q[:300])
+        with pytest.raises(dit3d.DitError) as e:
+            dit3d.dit_wait_device(60_000_000)
+        assert e.value.status == 7
+    finally:
+        dit3d.lib().dit_debug_force_timeout(0)
+    dit3d.dit_wait_device(60_000_000)

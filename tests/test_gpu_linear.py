@@ -102,6 +102,26 @@ def test_linear_bounded_wait_reports_timeout(variant):
     assert (o.float() - ref).abs().max().item() < 0.5
 
 
+def test_linear_wait_that_runs_out_reports_timeout():
+    # single-CTA GEMM with a wait limit of 1 ns: a wait runs out mid-pipeline
+    g = torch.Generator(device="cuda").manual_seed(9)
+    x = torch.randn(4096, 2048, device="cuda", generator=g).to(torch.bfloat16)
+    w = torch.randn(4096, 2048, device="cuda", generator=g).to(torch.bfloat16)
+    ref = dit3d.dit_linear(x, w)
+    dit3d.dit_check_device()
+    dit3d.lib().dit_debug_wait_limit_ns(1)
+    try:
+        dit3d.dit_linear(x, w)
+        with pytest.raises(dit3d.DitError) as e:
+            dit3d.dit_check_device()
+        assert e.value.status == 7
+    finally:
+        dit3d.lib().dit_debug_wait_limit_ns(0)
+    o = dit3d.dit_linear(x, w)
+    dit3d.dit_check_device()
+    assert torch.equal(o, ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 208), (1000, 1024, 512), (77, 3072, 144)])
 @pytest.mark.parametrize("mode", ["plain", "bias_gelu", "gated"])
 def test_linear_fp8_parity(M, N, K, mode):

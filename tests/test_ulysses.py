@@ -151,3 +151,67 @@ def test_varlen_sequences_placed_by_lpt_give_the_packed_result(world):
     assert placed == list(range(len(lens)))                 # every sequence exactly once
     for rank, err, _ in res:
         assert err == 0.0, f"rank {rank}: gathered output differs from the packed batch by {err}"
+
+
+def _oracle_attend(rope):
+    """The chunk compute of ulysses_attention with the fp64 oracle in place of the
+    kernels (RoPE on the whole packed sequences, then attention per sequence)."""
+    def attend(qh, kh, vh, layout):
+        cu = np.asarray(layout.cu, np.int32)
+        qr = oracle.rope3d(qh.numpy(), cu, rope["grid_h"], rope["grid_w"], rope["bands"])
+        kr = oracle.rope3d(kh.numpy(), cu, rope["grid_h"], rope["grid_w"], rope["bands"])
+        oh, _ = oracle.attn_fwd(qr, kr, vh.numpy(), cu)
+        return torch.from_numpy(np.ascontiguousarray(oh))
+    return attend
+
+
+def _chunked_worker(rank, world, port, q, lens, H, d, grid, chunks):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        Q, K, V = _full(int(cu[-1]), H, d, 11)
+        layout = ulysses.UlyssesLayout(cu, world)
+        mine = layout.local_rows(rank).numpy()
+        rope = dict(grid_h=grid[0], grid_w=grid[1], bands=(d // 4, d // 4 + d // 8, d // 2 - d // 8))
+        o = ulysses.ulysses_attention(*(torch.from_numpy(np.ascontiguousarray(t[mine]))
+                                        for t in (Q, K, V)),
+                                      cu_seqlens=cu, head_chunks=chunks,
+                                      attend=_oracle_attend(rope))
+        ref, _ = oracle.attn_fwd(Q, K, V, cu, qrows=mine, rope=dict(rope, base=10000.0))
+        q.put((rank, float(np.abs(o.numpy() - ref).max())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,lens,chunks", [(2, [96], 2), (2, [48, 24, 72], 2), (4, [96, 48], 2),
+                                              (4, [24, 96], 1)])
+def test_chunked_ulysses_on_packed_batches_equals_the_unsplit_attention(world, lens, chunks):
+    # 4x6 patch frames; each sequence's length a multiple of the rank count; this rank's
+    # heads in `chunks` chunks whose exchanges overlap the previous chunk's attention
+    H, d, grid = 8, 16, (4, 6)
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_chunked_worker, args=(r, world, port, q, lens, H, d, grid, chunks))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err in res:
+        assert err < 1e-12, f"rank {rank}: chunked split attention differs by {err}"
+
+
+def test_ulysses_layout_places_every_row_once():
+    lay = ulysses.UlyssesLayout([0, 8, 20], 2)
+    assert lay.rows_local == 10
+    assert lay.local_rows(0).tolist() == [0, 1, 2, 3, 8, 9, 10, 11, 12, 13]
+    assert lay.local_rows(1).tolist() == [4, 5, 6, 7, 14, 15, 16, 17, 18, 19]
+    # gather after the exchange undoes the rank-major order exactly
+    received = torch.cat([lay.local_rows(0), lay.local_rows(1)])
+    assert received.index_select(0, lay.gather_idx).tolist() == list(range(20))
+    with pytest.raises(ValueError):
+        ulysses.UlyssesLayout([0, 9], 2)
