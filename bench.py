@@ -39,11 +39,11 @@ sys.path.insert(0, ROOT)
 METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
 UNIT = "TFLOP/s"
 # DRAM bytes per head of one attention launch at the 480P geometry, from an ncu capture
-# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum over 16), keyed by RoPE mode
-# ("prepass" and "none" run the same kernel, without in-kernel RoPE). Heads are
-# independent, so a launch's traffic is this times its head count. None where the
-# current kernel has not been captured; other workloads report null.
-ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 526.166784e6 / 16, "none": 526.166784e6 / 16,
+# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum = 410.60 + 118.89 MB, over
+# 16), keyed by RoPE mode ("prepass" and "none" run the same kernel, without in-kernel
+# RoPE). Heads are independent, so a launch's traffic is this times its head count.
+# None where the current kernel has not been captured; other workloads report null.
+ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 529.48736e6 / 16, "none": 529.48736e6 / 16,
                                  "fused": None}
 
 
