@@ -61,7 +61,7 @@ def test_workload_attention_sampled(case):
     o, lse = dit3d.dit_attn_fwd(q, k, v, n_seq=w.n_seq, cu_seqlens=cu if w.varlen else None,
                                 rope=desc, return_lse=True)
     dit3d.dit_check_device()
-    rows = wl.sample_rows(w, per_seq=64 if w.name in ("480p", "720p", "varlen") else 256)
+    rows = wl.sample_rows(w, per_seq=256)
     if w.name == "tiny":
         rows = np.arange(w.rows)
     ref_o, ref_lse = oracle.attn_fwd(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), cu,
