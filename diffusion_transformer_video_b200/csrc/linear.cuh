@@ -285,13 +285,12 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
 // tile with M = 256 MMAs issued by the even CTA. Each CTA loads its own 128 rows of A
 // and one half (128 rows) of the B tile, so a k-block costs each SM 32 KB of loads
 // instead of 48 KB, and the 6-stage ring holds more k-blocks in flight. Each CTA's
-// TMEM holds its 128 rows x 256 columns (two buffers). Readiness crosses the pair
-// through the even CTA's barriers: a relay thread in each CTA waits for its own
-// stage to land and arrives (release, cluster scope) on the even CTA's ready[s]; the
-// MMA commits arrive on both CTAs' barriers (multicast commit); the epilogue of each
-// CTA signals the even CTA's acc_empty[b] once its 128 threads have drained buffer b.
-// No load is multicast. Measured on B200 at the 480P projection shapes: 2.3x slower
-// than the single-CTA form (601 against 1401 TFLOP/s), so it is not the default.
+// TMEM holds its 128 rows x 256 columns (two buffers). Both CTAs' loads complete on
+// the even CTA's full[s] (cta_group::2 tensor loads; the even CTA's producer expects
+// both CTAs' bytes), which is all the MMA thread waits for; the MMA commits arrive on
+// both CTAs' barriers (multicast commit), so each producer waits for its own empty[s];
+// the epilogue of each CTA signals the even CTA's acc_empty[b] once its 128 threads
+// have drained buffer b. No load is multicast.
 constexpr int kStages2 = 6;
 constexpr int kGroupM2 = 8;                            // pair tiles (256 rows) per group
 constexpr uint32_t kHalfBytes = kBM * kBK * 2;         // 16 KB: A half or B half
@@ -319,8 +318,8 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ __align__(8) uint64_t full[kStages2], ready[kStages2], empty[kStages2], acc_full[2],
-      acc_empty[2], drain;
+  __shared__ __align__(8) uint64_t full[kStages2], empty[kStages2], acc_full[2], acc_empty[2],
+      drain;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -334,7 +333,6 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     s_abort = p.force_timeout ? 1 : 0;
     for (int s = 0; s < kStages2; ++s) {
       ptx::mbar_init(ptx::smem_u32(&full[s]), 1);
-      ptx::mbar_init(ptx::smem_u32(&ready[s]), 2);
       ptx::mbar_init(ptx::smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -377,33 +375,23 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
             ok = false;
             break;
           }
-          const uint32_t f = ptx::smem_u32(&full[s]);
+          // both CTAs' bytes land on the even CTA's full[s]
+          const uint32_t f_even = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
           const uint32_t dst = ptx::smem_u32(smem + s * kStageBytes2);
-          ptx::mbar_arrive_expect_tx(f, kStageBytes2);
-          ptx::tma_load_2d(dst, &tm_a, kb * kBK, ya, f);
-          ptx::tma_load_2d(dst + kHalfBytes, &tm_b, kb * kBK, yb, f);
+          if (leader) ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), 2 * kStageBytes2);
+          ptx::tma_load_2d_pair(dst, &tm_a, kb * kBK, ya, f_even);
+          ptx::tma_load_2d_pair(dst + kHalfBytes, &tm_b, kb * kBK, yb, f_even);
         }
       }
-      volatile int never = 0;
-      for (int j = (it > kStages2 ? it - kStages2 : 0); j < it; ++j)
-        ptx::mbar_wait(ptx::smem_u32(&full[j % kStages2]), (j / kStages2) & 1, &never);
-    }
-    __syncwarp();
-  } else if (warp == 2) {
-    // ================================================================ relay
-    // this CTA's stage landed -> one arrival on the even CTA's ready[s]
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int t = cluster; ok && t < n_tiles; t += n_clusters)
-        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
-          const int s = it % kStages2;
-          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages2) & 1, abort)) {
-            ok = false;
-            break;
-          }
-          arrive_leader(&ready[s]);
-        }
+      // no copy may still be in flight into either CTA's shared memory when the pair
+      // exits: the even CTA's full[s] counts both CTAs' bytes, and both producers issue
+      // the same stages (each waits for the same multicast commits), so the even CTA
+      // waits for them and the cluster barrier at the end holds the odd CTA until then
+      if (leader) {
+        volatile int never = 0;
+        for (int j = (it > kStages2 ? it - kStages2 : 0); j < it; ++j)
+          ptx::mbar_wait(ptx::smem_u32(&full[j % kStages2]), (j / kStages2) & 1, &never);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -423,7 +411,7 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         ptx::tc_fence_after();
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % kStages2;
-          if (!ptx::mbar_wait_cluster(ptx::smem_u32(&ready[s]), (it / kStages2) & 1, abort)) {
+          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages2) & 1, abort)) {
             ok = false;
             break;
           }
