@@ -109,10 +109,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^t of a pair of scores on the MUFU unit (ex2.approx). Moving a share of these to
-// an FMA-pipe polynomial (Cody-Waite reduction, degree-3 minimax) was measured slower
-// on B200 (a quarter of the pairs: -7 %; half: -15 %): the softmax warp's issue, not
-// the MUFU rate, sets its pace.
+// 2^t of a pair of scores on the MUFU unit (ex2.approx; 16 results per clock per SM
+// on B200, and the packed f16x2 / bf16x2 forms give no more). Moving a share of these
+// to the FMA pipe (rounding by adding 1.5 * 2^23, degree-3 minimax polynomial for 2^f,
+// 2^j added to the exponent field: no conversion instruction, which would issue to the
+// MUFU pipe as well) was measured slower on B200: a quarter of the pairs -3 to -5 %,
+// three eighths or half -12 to -17 %. The MUFU rate does not set the softmax's pace.
 __device__ __forceinline__ void exp2_pair(uint64_t t2, float& e0, float& e1) {
   float t0, t1;
   f2_unpack(t2, t0, t1);
@@ -329,8 +331,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(ptx::smem_u32(&b->s_full[i]), 1);
-      ptx::mbar_init(ptx::smem_u32(&b->p_half[i]), kTileM);
-      ptx::mbar_init(ptx::smem_u32(&b->p_full[i]), kTileM);
+      // one arrival per softmax warp: measured 4 % faster at 480P than one per thread
+      ptx::mbar_init(ptx::smem_u32(&b->p_half[i]), kTileM / 32);
+      ptx::mbar_init(ptx::smem_u32(&b->p_full[i]), kTileM / 32);
     }
     ptx::mbar_init(ptx::smem_u32(&b->o_final), 1);
     ptx::mbar_init(ptx::smem_u32(&b->drain), 1);
@@ -435,14 +438,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         else ptx::tmem_st16(tS + 16 * q4, pw);
         if (q4 == 1) {
           // keys 0-63 are in TMEM: the MMA warp may start O += P V on them
+          // (every lane's stores complete and fenced, then one arrival for the warp)
           ptx::tmem_wait_st();
           ptx::tc_fence_before();
-          ptx::mbar_arrive(bar_ph);
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar_ph);
         }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar_p);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_p);
     }
     // ---- epilogue: O / l -> bf16 -> global, plus the log-sum-exp
     if (__all_sync(0xffffffffu, ok && ptx::mbar_wait(ptx::smem_u32(&b->o_final), 0, abort, p.wait_limit_ns))) {
@@ -524,7 +530,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncwarp();
   } else if (warp == kWarpMma) {
     // =========================================================== MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop, so control flow and every operand are
+    // warp-uniform, and one elected lane issues each tcgen05 instruction. Measured on
+    // B200: with a single lane running the loop, a key step (32 MMAs of 64 clocks) took
+    // ~3,600 clocks while no wait found its barrier incomplete, i.e. issue, not data,
+    // set the pace; the whole-warp form is 6-12 % faster on every workload, same bits.
+    {
+      const bool leader = ptx::elect_one();
+      // every lane waits; the result is made warp-uniform
+      auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, p.wait_limit_ns));
+      };
       constexpr uint32_t idesc_qk = ptx::make_idesc_bf16_f32(kTileM, kTileN, false);
       constexpr uint32_t idesc_pv = ptx::make_idesc_bf16_f32(kTileM, D, true);
       const uint32_t sbase = ptx::smem_u32(smem);
@@ -536,7 +552,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           constexpr uint32_t idesc_qk8 = ptx::make_idesc_e4m3_f32(kTileM, kTileN);
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)  // 32 bytes = 32 E4M3 elements per MMA
-            ptx::umma_ss_f8(tmem + col_s(qi),
+            if (leader) ptx::umma_ss_f8(tmem + col_s(qi),
                             ptx::make_smem_desc(qa + kk * 32, 16, 1024, ptx::kSwizzle128B),
                             ptx::make_smem_desc(ka + kk * 32, 16, 1024, ptx::kSwizzle128B),
                             idesc_qk8, kk > 0);
@@ -544,12 +560,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            ptx::umma_ss(tmem + col_s(qi), ptx::make_smem_desc(qa + off, 16, 1024, ptx::kSwizzle128B),
+            if (leader) ptx::umma_ss(tmem + col_s(qi), ptx::make_smem_desc(qa + off, 16, 1024, ptx::kSwizzle128B),
                          ptx::make_smem_desc(ka + off, 16, 1024, ptx::kSwizzle128B), idesc_qk,
                          kk > 0);
           }
         }
-        ptx::umma_commit(ptx::smem_u32(&b->s_full[qi]));
+        if (leader) ptx::umma_commit(ptx::smem_u32(&b->s_full[qi]));
       };
       // O_qi (+)= P_qi V over keys [64 * half, 64 * half + 64)
       auto pv = [&](int qi, int st, bool acc, int half) {
@@ -560,7 +576,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int k2 = 0; k2 < kTileN / 64; ++k2) {
             const int kk = half * (kTileN / 64) + k2;
-            ptx::umma_ts_f8(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
+            if (leader) ptx::umma_ts_f8(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
                             ptx::make_smem_desc(va + kk * 4096, 16384, 1024, ptx::kSwizzle128B),
                             idesc_pv8, (acc || kk > 0) ? 1u : 0u);
           }
@@ -568,7 +584,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int k4 = 0; k4 < kTileN / 32; ++k4) {
             const int kk = half * (kTileN / 32) + k4;
-            ptx::umma_ts(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
+            if (leader) ptx::umma_ts(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
                          ptx::make_smem_desc(va + kk * 2048, 16384, 1024, ptx::kSwizzle128B),
                          idesc_pv, (acc || kk > 0) ? 1u : 0u);
           }
@@ -576,49 +592,47 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
       // both halves, the second once the softmax has stored all of P
       auto pv_tile = [&](int qi, int st, bool acc, int j) -> bool {
-        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_half[qi]), j & 1, abort, p.wait_limit_ns)) return false;
+        if (!wait(ptx::smem_u32(&b->p_half[qi]), j & 1)) return false;
         ptx::tc_fence_after();
         pv(qi, st, acc, 0);
-        if (!ptx::mbar_wait(ptx::smem_u32(&b->p_full[qi]), j & 1, abort, p.wait_limit_ns)) return false;
+        if (!wait(ptx::smem_u32(&b->p_full[qi]), j & 1)) return false;
         ptx::tc_fence_after();
         pv(qi, st, acc, 1);
         return true;
       };
       const uint32_t q_wait = ptx::smem_u32(p.use_rope ? &b->q_ready : &b->q_full);
-      bool ok = ptx::mbar_wait(q_wait, 0, abort, p.wait_limit_ns);
-      if (ok) ok = ptx::mbar_wait(ptx::smem_u32(p.use_rope ? &b->k_ready[0] : &b->k_full[0]), 0, abort, p.wait_limit_ns);
+      bool ok = wait(q_wait, 0);
+      if (ok) ok = wait(ptx::smem_u32(p.use_rope ? &b->k_ready[0] : &b->k_full[0]), 0);
       if (ok) {
         ptx::tc_fence_after();
         qk(0, 0);
         qk(1, 0);
-        ptx::umma_commit(ptx::smem_u32(&b->k_empty[0]));
+        if (leader) ptx::umma_commit(ptx::smem_u32(&b->k_empty[0]));
         issued_any = true;
       }
       for (int j = 0; ok && j < nk; ++j) {
         const int vs = j % kVStages, vph = (j / kVStages) & 1;
         const int ks1 = (j + 1) % kKStages, kph1 = ((j + 1) / kKStages) & 1;
         const bool more = j + 1 < nk;
-        if (!(ok = ptx::mbar_wait(ptx::smem_u32(&b->v_full[vs]), vph, abort, p.wait_limit_ns))) break;
+        if (!(ok = wait(ptx::smem_u32(&b->v_full[vs]), vph))) break;
         if (!(ok = pv_tile(0, vs, j > 0, j))) break;
         if (more) {
-          if (!(ok = ptx::mbar_wait(
-                    ptx::smem_u32(p.use_rope ? &b->k_ready[ks1] : &b->k_full[ks1]), kph1, abort, p.wait_limit_ns)))
-            break;
+          if (!(ok = wait(ptx::smem_u32(p.use_rope ? &b->k_ready[ks1] : &b->k_full[ks1]), kph1))) break;
           ptx::tc_fence_after();
           qk(0, ks1);
         }
         if (!(ok = pv_tile(1, vs, j > 0, j))) break;
-        ptx::umma_commit(ptx::smem_u32(&b->v_empty[vs]));
+        if (leader) ptx::umma_commit(ptx::smem_u32(&b->v_empty[vs]));
         if (more) {
           qk(1, ks1);
-          ptx::umma_commit(ptx::smem_u32(&b->k_empty[ks1]));
+          if (leader) ptx::umma_commit(ptx::smem_u32(&b->k_empty[ks1]));
         }
       }
-      if (ok) ptx::umma_commit(ptx::smem_u32(&b->o_final));
+      if (ok && leader) ptx::umma_commit(ptx::smem_u32(&b->o_final));
       if (issued_any) {
         // all MMAs of this CTA complete before tensor memory is released
         volatile int never = 0;
-        ptx::umma_commit(ptx::smem_u32(&b->drain));
+        if (leader) ptx::umma_commit(ptx::smem_u32(&b->drain));
         ptx::mbar_wait(ptx::smem_u32(&b->drain), 0, &never);
       }
     }

@@ -63,11 +63,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait on phase `parity` of an mbarrier. Gives up after `limit_ns`
 // of wall time, or as soon as another role of the CTA raised `*abort`; both are
-// checked after the first unsuccessful try and then every 256 tries.
+// checked after the second unsuccessful try and then every 256 tries. The first
+// blocking try comes before the timer is read, so a phase that completes while the
+// thread is suspended in it is seen at once.
 // Returns false when it gave up; the caller must then leave its loop.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
   if (mbar_test_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -93,11 +96,25 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Same contract as mbar_wait, with acquire at cluster scope; the fast path is a
+// non-blocking probe, as in mbar_wait.
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort,
                                                   uint64_t limit_ns = 2000000000ull) {
+  if (mbar_test_wait_cluster(bar, parity)) return true;
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort) return false;
@@ -107,6 +124,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
       }
     }
   }
+}
+// One lane of the (converged) warp: true there, false on the other 31 lanes.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r));
+  return r != 0;
 }
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
