@@ -413,7 +413,12 @@ attn_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else if (warp == kWarpMma) {
     // =========================================================== MMA issuer (even CTA)
-    if (leader && lane == 0) {
+    // whole warp, one elected lane issuing (warp-uniform control flow and operands)
+    if (leader) {
+      const bool issuer = ptx::elect_one();
+      auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, ptx::mbar_wait_cluster(bar, parity, abort));
+      };
       constexpr uint32_t idesc_qk = ptx::make_idesc_bf16_f32(256, kTileN, false);
       constexpr uint32_t idesc_pv = ptx::make_idesc_bf16_f32(256, kD, true);
       const uint32_t sbase = ptx::smem_u32(smem);
@@ -423,64 +428,64 @@ attn_fwd_2sm_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t ka = sbase + L::kK + sl * L::kKSlot;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk)
-          ptx::umma_ss_pair(tmem + col_s(qi),
+          if (issuer) ptx::umma_ss_pair(tmem + col_s(qi),
                             ptx::make_smem_desc(qa + (kk >> 2) * L::kQBlock + (kk & 3) * 32, 16,
                                                 1024, ptx::kSwizzle128B),
                             ptx::make_smem_desc(ka + (kk >> 2) * L::kKBlock + (kk & 3) * 32, 16,
                                                 1024, ptx::kSwizzle128B),
                             idesc_qk, kk > 0);
-        ptx::umma_commit_pair(ptx::smem_u32(&b->s_full[qi]));
+        if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&b->s_full[qi]));
       };
       auto pv = [&](int qi, int sl, bool acc, int half) {
         const uint32_t va = sbase + L::kV + sl * L::kVSlot;
 #pragma unroll
         for (int k4 = 0; k4 < kTileN / 32; ++k4) {
           const int kk = half * (kTileN / 32) + k4;
-          ptx::umma_ts_pair(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
+          if (issuer) ptx::umma_ts_pair(tmem + col_o(qi), tmem + col_s(qi) + kk * 8,
                             ptx::make_smem_desc(va + kk * 2048, L::kVSlot, 1024, ptx::kSwizzle128B),
                             idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
       };
       auto pv_tile = [&](int qi, int sl, bool acc, int j) -> bool {
-        if (!ptx::mbar_wait_cluster(ptx::smem_u32(&b->p_half[qi]), j & 1, abort)) return false;
+        if (!wait(ptx::smem_u32(&b->p_half[qi]), j & 1)) return false;
         ptx::tc_fence_after();
         pv(qi, sl, acc, 0);
-        if (!ptx::mbar_wait_cluster(ptx::smem_u32(&b->p_full[qi]), j & 1, abort)) return false;
+        if (!wait(ptx::smem_u32(&b->p_full[qi]), j & 1)) return false;
         ptx::tc_fence_after();
         pv(qi, sl, acc, 1);
         return true;
       };
-      bool ok = ptx::mbar_wait_cluster(ptx::smem_u32(&b->q_ready), 0, abort);
-      if (ok) ok = ptx::mbar_wait_cluster(ptx::smem_u32(&b->k_ready[0]), 0, abort);
+      bool ok = wait(ptx::smem_u32(&b->q_ready), 0);
+      if (ok) ok = wait(ptx::smem_u32(&b->k_ready[0]), 0);
       if (ok) {
         ptx::tc_fence_after();
         qk(0, 0);
         qk(1, 0);
-        ptx::umma_commit_pair(ptx::smem_u32(&b->k_empty[0]));
+        if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&b->k_empty[0]));
         issued_any = true;
       }
       for (int j = 0; ok && j < nk; ++j) {
         const int sl = j % kSlots, ph = (j / kSlots) & 1;
         const int sl1 = (j + 1) % kSlots, ph1 = ((j + 1) / kSlots) & 1;
         const bool more = j + 1 < nk;
-        if (!(ok = ptx::mbar_wait_cluster(ptx::smem_u32(&b->v_ready[sl]), ph, abort))) break;
+        if (!(ok = wait(ptx::smem_u32(&b->v_ready[sl]), ph))) break;
         if (!(ok = pv_tile(0, sl, j > 0, j))) break;
         if (more) {
-          if (!(ok = ptx::mbar_wait_cluster(ptx::smem_u32(&b->k_ready[sl1]), ph1, abort))) break;
+          if (!(ok = wait(ptx::smem_u32(&b->k_ready[sl1]), ph1))) break;
           ptx::tc_fence_after();
           qk(0, sl1);
         }
         if (!(ok = pv_tile(1, sl, j > 0, j))) break;
-        ptx::umma_commit_pair(ptx::smem_u32(&b->v_empty[sl]));
+        if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&b->v_empty[sl]));
         if (more) {
           qk(1, sl1);
-          ptx::umma_commit_pair(ptx::smem_u32(&b->k_empty[sl1]));
+          if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&b->k_empty[sl1]));
         }
       }
-      if (ok) ptx::umma_commit_pair(ptx::smem_u32(&b->o_final));
+      if (ok && issuer) ptx::umma_commit_pair(ptx::smem_u32(&b->o_final));
       if (issued_any) {
         volatile int never = 0;
-        ptx::umma_commit_pair(ptx::smem_u32(&b->drain));
+        if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&b->drain));
         ptx::mbar_wait_cluster(ptx::smem_u32(&b->drain), 0, &never);
       }
     }

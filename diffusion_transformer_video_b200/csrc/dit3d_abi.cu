@@ -33,7 +33,7 @@ namespace {
 std::mutex g_mu;
 int g_force_timeout = 0;
 uint64_t g_wait_limit_ns = 2000000000ull;  // bound of the single-CTA kernels' waits
-int g_linear_variant = 0;  // 0: one CTA per 128x256 tile; 1: CTA pairs per 256x256 tile
+int g_linear_variant = 1;  // 1 (default): CTA pairs per 256x256 tile; 0: one CTA per 128x256 tile
 int g_attn_variant = 0;  // 0: one CTA per query-tile pair; 1: CTA pairs (head_dim 128)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -187,22 +187,27 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
     __syncwarp();
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform control flow and operands); one
+    // elected lane issues each tcgen05 instruction.
+    {
+      const bool leader = ptx::elect_one();
+      auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort, p.wait_limit_ns));
+      };
       constexpr uint32_t idesc = ptx::make_idesc_bf16_f32(kBM, kBN, false);
       int it = 0, local = 0;
       bool ok = true, issued = false;
       for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++local) {
         const int b = local & 1;
         const uint32_t acc = tmem + static_cast<uint32_t>(b * kBN);
-        if (local >= 2 &&
-            !ptx::mbar_wait(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1, abort, p.wait_limit_ns)) {
+        if (local >= 2 && !wait(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % kStages;
-          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages) & 1, abort, p.wait_limit_ns)) {
+          if (!wait(ptx::smem_u32(&full[s]), (it / kStages) & 1)) {
             ok = false;
             break;
           }
@@ -213,22 +218,23 @@ linear_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ 
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t da = ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B);
             const uint64_t db = ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B);
+            if (!leader) continue;
             if constexpr (F8)
               ptx::umma_ss_f8(acc, da, db, ptx::make_idesc_e4m3_f32(kBM, kBN),
                               (kb > 0 || kk > 0) ? 1u : 0u);
             else
               ptx::umma_ss(acc, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          ptx::umma_commit(ptx::smem_u32(&empty[s]));
+          if (leader) ptx::umma_commit(ptx::smem_u32(&empty[s]));
           issued = true;
         }
         if (!ok) break;
-        ptx::umma_commit(ptx::smem_u32(&acc_full[b]));
+        if (leader) ptx::umma_commit(ptx::smem_u32(&acc_full[b]));
       }
       if (issued) {
         // every MMA of this CTA completes before tensor memory is released
         volatile int never = 0;
-        ptx::umma_commit(ptx::smem_u32(&drain));
+        if (leader) ptx::umma_commit(ptx::smem_u32(&drain));
         ptx::mbar_wait(ptx::smem_u32(&drain), 0, &never);
       }
     }
@@ -396,7 +402,9 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     __syncwarp();
   } else if (warp == 1) {
     // ================================================================ MMA issuer (even CTA)
-    if (leader && lane == 0) {
+    // whole warp, one elected lane issuing (as in the single-CTA kernel)
+    if (leader) {
+      const bool issuer = ptx::elect_one();
       constexpr uint32_t idesc = ptx::make_idesc_bf16_f32(2 * kBM, kBN, false);
       int it = 0, local = 0;
       bool ok = true, issued = false;
@@ -404,14 +412,15 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         const int b = local & 1;
         const uint32_t acc = tmem + static_cast<uint32_t>(b * kBN);
         if (local >= 2 &&
-            !ptx::mbar_wait_cluster(ptx::smem_u32(&acc_empty[b]), ((local / 2) - 1) & 1, abort)) {
+            !__all_sync(0xffffffffu, ptx::mbar_wait_cluster(ptx::smem_u32(&acc_empty[b]),
+                                                            ((local / 2) - 1) & 1, abort))) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = it % kStages2;
-          if (!ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages2) & 1, abort)) {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(ptx::smem_u32(&full[s]), (it / kStages2) & 1, abort))) {
             ok = false;
             break;
           }
@@ -419,18 +428,19 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           const uint32_t a0 = ptx::smem_u32(smem + s * kStageBytes2), b0 = a0 + kHalfBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            ptx::umma_ss_pair(acc, ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B),
-                              ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B), idesc,
-                              (kb > 0 || kk > 0) ? 1u : 0u);
-          ptx::umma_commit_pair(ptx::smem_u32(&empty[s]));
+            if (issuer)
+              ptx::umma_ss_pair(acc, ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B),
+                                ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B), idesc,
+                                (kb > 0 || kk > 0) ? 1u : 0u);
+          if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&empty[s]));
           issued = true;
         }
         if (!ok) break;
-        ptx::umma_commit_pair(ptx::smem_u32(&acc_full[b]));
+        if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&acc_full[b]));
       }
       if (issued) {
         volatile int never = 0;
-        ptx::umma_commit_pair(ptx::smem_u32(&drain));
+        if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&drain));
         ptx::mbar_wait_cluster(ptx::smem_u32(&drain), 0, &never);
       }
     }

@@ -11,6 +11,7 @@ from tests.helpers import check_modulation, f64, from_dev, to_dev
 
 pytestmark = pytest.mark.gpu
 RNG = np.random.default_rng(31)
+DEFAULT_VARIANT = 1  # CTA pairs
 
 
 def bits(shape, std=1.0):
@@ -21,7 +22,7 @@ def bits(shape, std=1.0):
 def variant(request):
     dit3d.dit_set_linear_variant(request.param)
     yield request.param
-    dit3d.dit_set_linear_variant(0)
+    dit3d.dit_set_linear_variant(DEFAULT_VARIANT)
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (1, 8, 8), (300, 520, 200), (1000, 1024, 512),
@@ -76,7 +77,7 @@ def test_linear_variants_agree():
     for v in (0, 1):
         dit3d.dit_set_linear_variant(v)
         outs.append(dit3d.dit_linear(x, w))
-    dit3d.dit_set_linear_variant(0)
+    dit3d.dit_set_linear_variant(DEFAULT_VARIANT)
     dit3d.dit_check_device()
     # same products, fp32 sums in possibly different order: within one bf16 ulp
     diff = (outs[0].float() - outs[1].float()).abs()
@@ -103,23 +104,28 @@ def test_linear_bounded_wait_reports_timeout(variant):
 
 
 def test_linear_wait_that_runs_out_reports_timeout():
-    # single-CTA GEMM with a wait limit of 1 ns: a wait runs out mid-pipeline
+    # single-CTA GEMM with a wait limit of 1 ns: a wait runs out mid-pipeline (the CTA-pair
+    # form keeps its 2 s limit)
     g = torch.Generator(device="cuda").manual_seed(9)
     x = torch.randn(4096, 2048, device="cuda", generator=g).to(torch.bfloat16)
     w = torch.randn(4096, 2048, device="cuda", generator=g).to(torch.bfloat16)
-    ref = dit3d.dit_linear(x, w)
-    dit3d.dit_check_device()
-    dit3d.lib().dit_debug_wait_limit_ns(1)
+    dit3d.dit_set_linear_variant(0)
     try:
-        dit3d.dit_linear(x, w)
-        with pytest.raises(dit3d.DitError) as e:
-            dit3d.dit_check_device()
-        assert e.value.status == 7
+        ref = dit3d.dit_linear(x, w)
+        dit3d.dit_check_device()
+        dit3d.lib().dit_debug_wait_limit_ns(1)
+        try:
+            dit3d.dit_linear(x, w)
+            with pytest.raises(dit3d.DitError) as e:
+                dit3d.dit_check_device()
+            assert e.value.status == 7
+        finally:
+            dit3d.lib().dit_debug_wait_limit_ns(0)
+        o = dit3d.dit_linear(x, w)
+        dit3d.dit_check_device()
+        assert torch.equal(o, ref)
     finally:
-        dit3d.lib().dit_debug_wait_limit_ns(0)
-    o = dit3d.dit_linear(x, w)
-    dit3d.dit_check_device()
-    assert torch.equal(o, ref)
+        dit3d.dit_set_linear_variant(DEFAULT_VARIANT)
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 208), (1000, 1024, 512), (77, 3072, 144)])
