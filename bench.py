@@ -39,11 +39,11 @@ sys.path.insert(0, ROOT)
 METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
 UNIT = "TFLOP/s"
 # DRAM bytes per head of one attention launch at the 480P geometry, from an ncu capture
-# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum = 410.60 + 118.89 MB, over
+# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum = 406.48 + 117.93 MB, over
 # 16), keyed by RoPE mode ("prepass" and "none" run the same kernel, without in-kernel
 # RoPE). Heads are independent, so a launch's traffic is this times its head count.
 # None where the current kernel has not been captured; other workloads report null.
-ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 529.48736e6 / 16, "none": 529.48736e6 / 16,
+ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 524.411392e6 / 16, "none": 524.411392e6 / 16,
                                  "fused": None}
 
 
@@ -76,7 +76,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -108,12 +108,26 @@ class ClockSampler:
             os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [v for v in (num(r[1]) for r in rows) if v is not None]
+        watts = [v for v in (num(r[3]) for r in rows) if v is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        mask = 0
+        for r in rows:  # union of the active-reasons bitmasks (0x4: software power cap)
+            try:
+                mask |= int(r[4], 16)
+            except ValueError:
+                pass
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
-                "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": num(rows[0][2]),
+                "reasons": reasons, "active_mask": hex(mask),
+                "power_w": statistics.median(watts) if watts else None, "samples": len(rows)}
 
 
 def widen_qkv(inp):
@@ -600,31 +614,33 @@ def main():
             if gated:
                 kw.update(residual=dev["x"], alpha=alpha_g, rows_per_group=rpg, out=x_next)
             run_lin = lambda: dit3d.dit_linear(xin, wt, **kw)
+            run_cublas = lambda: torch.matmul(xin, wt.t())  # same product, no epilogue
             for _ in range(2):
                 run_lin()
-            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                     for _ in range(5)]
-            for a, b in pairs:
+                run_cublas()
+
+            def per_call(fn):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                run_lin()
+                for _ in range(5):
+                    fn()
                 b.record(stream)
-            torch.cuda.synchronize()
+                torch.cuda.synchronize()
+                return a.elapsed_time(b) / 5
+
+            # ours and cuBLAS interleaved over three rounds (clocks drift under the power
+            # cap), median per call of each
+            t_ours, t_cublas = [], []
+            for _ in range(3):
+                t_ours.append(per_call(run_lin))
+                t_cublas.append(per_call(run_cublas))
             dit3d.dit_check_device()
-            ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+            ms, ms_cublas = statistics.median(t_ours), statistics.median(t_cublas)
             fl = 2.0 * rows * n_out * k_in
-            # cuBLAS (torch.matmul) on the same product, no epilogue: context only
-            for _ in range(2):
-                torch.matmul(xin, wt.t())
-            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            c0.record(stream)
-            for _ in range(5):
-                torch.matmul(xin, wt.t())
-            c1.record(stream)
-            torch.cuda.synchronize()
-            ms_cublas = c0.elapsed_time(c1) / 5
             lin[name] = {"ms": ms, "TFLOP/s": fl / (ms * 1e-3) / 1e12, "shape": [rows, n_out, k_in],
                          "frac_burst": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
-                         "cublas_ms": ms_cublas, "in_step": False}
+                         "cublas_ms": ms_cublas, "timing": "median of 3 rounds of 5 calls, "
+                         "interleaved with cuBLAS", "in_step": False}
             if name == "linear_qkv":
                 # the same projection on E4M3 activations and weights (scales 1/16, 1/256)
                 x8 = dit3d.dit_quantize_e4m3(xin, 16.0)

@@ -44,3 +44,19 @@ def test_reference_arm_prints_one_json_line():
     assert line["config"] == bench.workload_config(bench.resolve_workload(_args(workload="tiny")), 1)
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_clock_summary_reports_reasons_power_and_the_active_mask(tmp_path):
+    # rows as nvidia-smi prints them: index, clocks.sm, clocks.max.sm, power.draw,
+    # reasons bitmask, then the four yes/no reason fields
+    p = tmp_path / "clk.csv"
+    p.write_text("0, 1965, 1965, 612.40, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+                 "0, 1590, 1965, 998.10, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+                 "0, 1605, 1965, 996.00, 0x0000000000000004, Not Active, Not Active, Not Active, Not Active\n"
+                 "0, [N/A], 1965, [N/A], [N/A], Not Active, Not Active, Not Active, Not Active\n")
+    c = bench.ClockSampler(0)
+    c.path = str(p)
+    s = c.summary()
+    assert s["sm_mhz"] == 1605 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["active_mask"] == "0x4"
+    assert s["power_w"] == 996.0 and s["samples"] == 4
