@@ -374,8 +374,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_s, j & 1, abort, p.wait_limit_ns))) { ok = false; break; }
       ptx::tc_fence_after();
       uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + c * 32, sr + c * 32);
+      ptx::tmem_ld64(tS, sr);
+      ptx::tmem_ld64(tS + 64, sr + 64);
       ptx::tmem_wait_ld();
       float s[128];
 #pragma unroll
