@@ -39,6 +39,7 @@
 // Every mbarrier wait is bounded; on expiry the CTA sets an error bit, drains its
 // in-flight copies and MMAs, frees its tensor memory and exits.
 #pragma once
+#include <type_traits>
 #include "common.cuh"
 #include "quant.cuh"
 #include "rope3d.cuh"
@@ -113,14 +114,49 @@ __device__ __forceinline__ float ex2(float x) {
 // on B200, and the packed f16x2 / bf16x2 forms give no more). Moving a share of these
 // to the FMA pipe (rounding by adding 1.5 * 2^23, degree-3 minimax polynomial for 2^f,
 // 2^j added to the exponent field: no conversion instruction, which would issue to the
-// MUFU pipe as well) was measured slower on B200: a quarter of the pairs -3 to -5 %,
-// three eighths or half -12 to -17 %. The MUFU rate does not set the softmax's pace.
+// MUFU pipe as well) was measured slower on B200 in the bf16 kernel: a quarter of the
+// pairs -3 to -5 %, three eighths or half -12 to -17 %. In the E4M3 modes, whose MMAs
+// take half the time, the MUFU pipe does set the pace: there three pairs in sixteen run
+// on the FMA pipe (exp2_pair_fma; measured 2-4 % faster in both E4M3 modes, while one in
+// four or more slowed the E4M3 Q K^T mode).
 __device__ __forceinline__ void exp2_pair(uint64_t t2, float& e0, float& e1) {
   float t0, t1;
   f2_unpack(t2, t0, t1);
   e0 = ex2(t0);
   e1 = ex2(t1);
 }
+
+// 2^t of a pair of scores on the FMA and integer pipes:
+//  - t = j + f with j = round(t): adding 1.5 * 2^23 (round to nearest) leaves j in the
+//    low mantissa bits, with no conversion instruction (those share the MUFU pipe);
+//  - 2^f for f in [-1/2, 1/2] by a degree-3 polynomial fitted by the Remez exchange for
+//    relative error (7.5e-5 in fp32 Horner form; P is then rounded to bf16 or E4M3);
+//  - 2^j enters as j << 23 added to the exponent field.
+// t is clamped to >= -126 so the exponent field cannot wrap: a score more than 126
+// below the running maximum then weighs about 2^-126 instead of 0. Masked (-inf) keys
+// never take this path (a ragged last tile keeps every exponential on the MUFU unit).
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+constexpr float kP0 = 0.9999280571937561f, kP1 = 0.6932609677314758f;
+constexpr float kP2 = 0.2426111251115799f, kP3 = 0.0551716685295105f;
+__device__ __forceinline__ void exp2_pair_fma(uint64_t t2, float& e0, float& e1) {
+  float t0, t1;
+  f2_unpack(t2, t0, t1);
+  const uint64_t tc = f2_pack(fmaxf(t0, -126.f), fmaxf(t1, -126.f));
+  const uint64_t r = f2_add(tc, f2_pack(kRound, kRound));    // j in the low bits
+  const uint64_t jf = f2_add(r, f2_pack(-kRound, -kRound));  // j, exact
+  const uint64_t f = f2_fma(jf, f2_pack(-1.f, -1.f), tc);    // t - j, exact
+  uint64_t q = f2_fma(f2_pack(kP3, kP3), f, f2_pack(kP2, kP2));
+  q = f2_fma(q, f, f2_pack(kP1, kP1));
+  q = f2_fma(q, f, f2_pack(kP0, kP0));
+  float q0, q1, r0, r1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(r, r0, r1);
+  e0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(r0) << 23));
+  e1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(r1) << 23));
+}
+// Pairs c of each 32-key chunk (bit c, c = 0..15) whose exponential runs on the FMA
+// pipe in the E4M3 modes: 3, 8 and 13.
+constexpr uint32_t kExpFmaMaskF8 = 0x2108u;
 
 // Byte offset of the 16-byte chunk `cc` (8 bf16) of row r inside a 128-row tile
 // stored as d/64 column blocks of [128 rows x 128 B] with the 128-byte TMA swizzle.
@@ -380,7 +416,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-      if (j == nk - 1 && last_valid < kTileN) {
+      const bool ragged = j == nk - 1 && last_valid < kTileN;
+      if (ragged) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= last_valid) s[c] = -INFINITY;
@@ -416,34 +453,45 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // p = 2^(s * scale * log2(e) - m): packed FFMA2 for the affine part, MUFU ex2,
       // packed FADD2 for the row sum
       const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-m, -m);
+      // FMA_MASK: the pairs whose exponential runs on the FMA pipe (compile-time)
+      auto store_p = [&](auto fma_mask) {
+        constexpr uint32_t FMA_MASK = decltype(fma_mask)::value;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        // P for 32 keys -> 16 packed bf16 columns (8 E4M3 columns), stored as soon as
-        // they are ready
-        uint32_t pw[16];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          // P for 32 keys -> 16 packed bf16 columns (8 E4M3 columns), stored as soon as
+          // they are ready
+          uint32_t pw[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint64_t t2 = f2_fma(f2_pack(s[32 * q4 + 2 * c], s[32 * q4 + 2 * c + 1]), sc2, nm2);
-          float e0, e1;
-          exp2_pair(t2, e0, e1);
-          l2 = f2_add(l2, f2_pack(e0, e1));
-          if constexpr (PV8) {
-            const uint32_t h = e4m3x2(e0, e1);
-            pw[c >> 1] = (c & 1) ? (pw[c >> 1] | (h << 16)) : h;
-          } else {
-            pw[c] = pack_bf16x2(e0, e1);
+          for (int c = 0; c < 16; ++c) {
+            const uint64_t t2 = f2_fma(f2_pack(s[32 * q4 + 2 * c], s[32 * q4 + 2 * c + 1]), sc2, nm2);
+            float e0, e1;
+            if ((FMA_MASK >> c) & 1u) exp2_pair_fma(t2, e0, e1);
+            else exp2_pair(t2, e0, e1);
+            l2 = f2_add(l2, f2_pack(e0, e1));
+            if constexpr (PV8) {
+              const uint32_t h = e4m3x2(e0, e1);
+              pw[c >> 1] = (c & 1) ? (pw[c >> 1] | (h << 16)) : h;
+            } else {
+              pw[c] = pack_bf16x2(e0, e1);
+            }
+          }
+          if constexpr (PV8) ptx::tmem_st8(tS + 8 * q4, pw);
+          else ptx::tmem_st16(tS + 16 * q4, pw);
+          if (q4 == 1) {
+            // keys 0-63 are in TMEM: the MMA warp may start O += P V on them
+            // (every lane's stores complete and fenced, then one arrival for the warp)
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_ph);
           }
         }
-        if constexpr (PV8) ptx::tmem_st8(tS + 8 * q4, pw);
-        else ptx::tmem_st16(tS + 16 * q4, pw);
-        if (q4 == 1) {
-          // keys 0-63 are in TMEM: the MMA warp may start O += P V on them
-          // (every lane's stores complete and fenced, then one arrival for the warp)
-          ptx::tmem_wait_st();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar_ph);
-        }
+      };
+      if constexpr (QK8) {
+        if (ragged) store_p(std::integral_constant<uint32_t, 0u>{});
+        else store_p(std::integral_constant<uint32_t, kExpFmaMaskF8>{});
+      } else {
+        store_p(std::integral_constant<uint32_t, 0u>{});
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();

@@ -784,6 +784,30 @@ int dit_wait_device(void* stream, int64_t timeout_us) {
   return (err & kDevErrTimeout) ? DIT_ERR_TIMEOUT : DIT_OK;
 }
 
+namespace {
+// exp2_pair_fma on pairs of an fp32 array (a lone last element is paired with itself)
+__global__ void exp2_fma_probe_kernel(const float* t, float* e, int64_t n) {
+  const int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float t0 = t[i], t1 = i + 1 < n ? t[i + 1] : t0;
+  float e0, e1;
+  attn::exp2_pair_fma(f2_pack(t0, t1), e0, e1);
+  e[i] = e0;
+  if (i + 1 < n) e[i + 1] = e1;
+}
+}  // namespace
+
+int dit_debug_exp2_fma(const float* t, float* out, int64_t n, void* stream) {
+  if (n < 0) return DIT_ERR_SHAPE;
+  if (n == 0) return DIT_OK;
+  if (t == nullptr || out == nullptr) return DIT_ERR_NULL;
+  const int64_t pairs = (n + 1) / 2;
+  if ((pairs + 255) / 256 >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
+  exp2_fma_probe_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0,
+                          static_cast<cudaStream_t>(stream)>>>(t, out, n);
+  return launch_status();
+}
+
 int dit_debug_poll_fake(int64_t busy_polls, int fail, int64_t timeout_us, int64_t* polls) {
   int64_t n = 0;
   const int s = poll_until(

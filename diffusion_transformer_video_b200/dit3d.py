@@ -27,7 +27,7 @@ EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "d
            "dit_rope3d_qk", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout",
-           "dit_debug_wait_limit_ns", "dit_wait_device", "dit_debug_poll_fake")
+           "dit_debug_wait_limit_ns", "dit_wait_device", "dit_debug_poll_fake", "dit_debug_exp2_fma")
 
 
 class DitError(RuntimeError):
@@ -91,6 +91,8 @@ def lib():
         L.dit_wait_device.restype = ctypes.c_int
         L.dit_debug_poll_fake.argtypes = [i64, ctypes.c_int, i64, ctypes.POINTER(i64)]
         L.dit_debug_poll_fake.restype = ctypes.c_int
+        L.dit_debug_exp2_fma.argtypes = [P, P, i64, P]
+        L.dit_debug_exp2_fma.restype = ctypes.c_int
         for name in ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
                      "dit_check_device"):
             getattr(L, name).restype = ctypes.c_int
@@ -341,6 +343,15 @@ def dit_wait_device(timeout_us: int):
     blocking synchronisation); raises DitError with DIT_ERR_TIMEOUT if it has not
     finished by then or if a kernel gave up a wait."""
     _check(lib().dit_wait_device(_stream(), int(timeout_us)))
+
+
+def dit_debug_exp2_fma(t):
+    """2^t (t: fp32 CUDA tensor) by the attention's FMA-pipe exponential (test hook)."""
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError("t must be a contiguous fp32 CUDA tensor")
+    out = torch.empty_like(t)
+    _check(lib().dit_debug_exp2_fma(_ptr(t), _ptr(out), t.numel(), _stream()))
+    return out
 
 
 def dit_shutdown():

@@ -270,6 +270,15 @@ int dit_wait_device(void* stream, int64_t timeout_us);
  * (may be NULL). Needs no GPU. */
 int dit_debug_poll_fake(int64_t busy_polls, int fail, int64_t timeout_us, int64_t* polls);
 
+/* Test hook of the attention's FMA-pipe exponential (the share of the E4M3 modes'
+ * softmax exponentials that does not run on the MUFU unit; no counterpart in the source
+ * pages): out[i] = 2^t[i] by the kernel's own routine (round-to-nearest split t = j + f
+ * with the 1.5 * 2^23 constant, degree-3 minimax polynomial for 2^f, j added to the
+ * exponent field; t clamped to >= -126). t, out: device fp32 arrays of n elements; runs
+ * on `stream`. Errors: DIT_ERR_SHAPE for n < 0, DIT_ERR_NULL for a null array when
+ * n > 0, DIT_ERR_LAUNCH on a CUDA error. */
+int dit_debug_exp2_fma(const float* t, float* out, int64_t n, void* stream);
+
 /* Human-readable name of a dit_status code (static string, never NULL). */
 const char* dit_status_string(int status);
 

@@ -337,3 +337,25 @@ def test_host_watchdog_returns_while_work_runs_then_reports_success():
     finally:
         dit3d.lib().dit_debug_force_timeout(0)
     dit3d.dit_wait_device(60_000_000)
+
+
+def test_fma_pipe_exp2_meets_its_error_bound():
+    # the E4M3 modes' FMA-pipe exponential against 2^t in fp64: the degree-3 minimax of 2^f
+    # on [-1/2, 1/2] has relative error 7.5e-5 (Remez exchange), the split t = j + f and
+    # the exponent insertion are exact
+    t = torch.cat([torch.linspace(-125.9, 8.0, 400001), torch.arange(-125, 9).float(),
+                   torch.tensor([-0.5, 0.5, -1.5, 2.5, 7.999, -125.5, 0.0, 1e-7, -1e-7])]).cuda()
+    e = dit3d.dit_debug_exp2_fma(t).double().cpu().numpy()
+    ref = np.exp2(t.double().cpu().numpy())
+    rel = np.abs(e / ref - 1.0)
+    assert rel.max() <= 8e-5, (rel.max(), t.cpu().numpy()[rel.argmax()])
+    # at t = -126 the result is subnormal (within 2e-4); below it the input is clamped:
+    # positive and at most 2^-125
+    at = dit3d.dit_debug_exp2_fma(torch.tensor([-126.0], device="cuda")).double().item()
+    assert abs(at / 2.0 ** -126 - 1.0) <= 2e-4
+    lo = dit3d.dit_debug_exp2_fma(torch.tensor([-126.7, -200.0, -1e30, float("-inf")],
+                                               device="cuda")).double().cpu().numpy()
+    assert (lo > 0).all() and (lo <= 2.0 ** -125).all()
+    # odd length: the lone last element is evaluated too
+    odd = dit3d.dit_debug_exp2_fma(torch.tensor([1.0, 2.0, 3.0], device="cuda")).double().cpu().numpy()
+    np.testing.assert_allclose(odd, [2.0, 4.0, 8.0], rtol=8e-5)
