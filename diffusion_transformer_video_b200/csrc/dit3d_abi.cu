@@ -508,20 +508,25 @@ static int linear_impl(const void* x, const void* w, const void* bias, void* out
   const int64_t tiles = static_cast<int64_t>(prm.tiles_m) * prm.tiles_n;
   if (tiles >= (int64_t(1) << 31)) return DIT_ERR_SHAPE;
   if (sms <= 0) sms = 148;
-  if (g_linear_variant == 1 && !f8) {
+  if (g_linear_variant == 1) {
     // CTA pairs: 256 x 256 tiles, each CTA loads 128 rows of A and of B
     CUtensorMap tb2;
-    if (!make_tmap(&tb2, w, N, K, lin::kBM)) return DIT_ERR_LAUNCH;
-    static bool attr2_set[64] = {};
-    if (dev < 64 && !attr2_set[dev]) {
-      if (cudaFuncSetAttribute(lin::linear_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(lin::kSmemBytes2)) != cudaSuccess)
-        return DIT_ERR_LAUNCH;
-      attr2_set[dev] = true;
+    if (!(f8 ? make_tmap8(&tb2, w, N, K, lin::kBM) : make_tmap(&tb2, w, N, K, lin::kBM)))
+      return DIT_ERR_LAUNCH;
+    static bool attr2_set[2][64] = {};
+    if (dev < 64 && !attr2_set[f8][dev]) {
+      const cudaError_t e =
+          f8 ? cudaFuncSetAttribute(lin::linear_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(lin::kSmemBytes2))
+             : cudaFuncSetAttribute(lin::linear_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(lin::kSmemBytes2));
+      if (e != cudaSuccess) return DIT_ERR_LAUNCH;
+      attr2_set[f8][dev] = true;
     }
     const int64_t pair_tiles = static_cast<int64_t>((prm.tiles_m + 1) / 2) * prm.tiles_n;
     const unsigned grid = 2u * static_cast<unsigned>(std::min<int64_t>(pair_tiles, sms / 2));
-    lin::linear_pair_kernel<<<grid, lin::kThreads, lin::kSmemBytes2, st>>>(ta, tb2, prm);
+    if (f8) lin::linear_pair_kernel<true><<<grid, lin::kThreads, lin::kSmemBytes2, st>>>(ta, tb2, prm);
+    else lin::linear_pair_kernel<false><<<grid, lin::kThreads, lin::kSmemBytes2, st>>>(ta, tb2, prm);
     return launch_status();
   }
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, sms));

@@ -318,9 +318,13 @@ __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// F8: E4M3 x and w, 128 elements of K per 128-byte stage row, kind::f8f6f4 MMAs (as in
+// the single-CTA kernel).
+template <bool F8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const Params p) {
+  constexpr int kKPerStage = F8 ? 128 : kBK;  // elements of K per 128-byte row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -385,8 +389,8 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           const uint32_t f_even = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
           const uint32_t dst = ptx::smem_u32(smem + s * kStageBytes2);
           if (leader) ptx::mbar_arrive_expect_tx(ptx::smem_u32(&full[s]), 2 * kStageBytes2);
-          ptx::tma_load_2d_pair(dst, &tm_a, kb * kBK, ya, f_even);
-          ptx::tma_load_2d_pair(dst + kHalfBytes, &tm_b, kb * kBK, yb, f_even);
+          ptx::tma_load_2d_pair(dst, &tm_a, kb * kKPerStage, ya, f_even);
+          ptx::tma_load_2d_pair(dst + kHalfBytes, &tm_b, kb * kKPerStage, yb, f_even);
         }
       }
       // no copy may still be in flight into either CTA's shared memory when the pair
@@ -405,7 +409,8 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
     // whole warp, one elected lane issuing (as in the single-CTA kernel)
     if (leader) {
       const bool issuer = ptx::elect_one();
-      constexpr uint32_t idesc = ptx::make_idesc_bf16_f32(2 * kBM, kBN, false);
+      constexpr uint32_t idesc = F8 ? ptx::make_idesc_e4m3_f32(2 * kBM, kBN)
+                                    : ptx::make_idesc_bf16_f32(2 * kBM, kBN, false);
       int it = 0, local = 0;
       bool ok = true, issued = false;
       for (int t = cluster; ok && t < n_tiles; t += n_clusters, ++local) {
@@ -426,12 +431,15 @@ linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
           }
           ptx::tc_fence_after();
           const uint32_t a0 = ptx::smem_u32(smem + s * kStageBytes2), b0 = a0 + kHalfBytes;
+          // four MMAs of 32 bytes of K each (16 bf16 or 32 E4M3 elements)
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            if (issuer)
-              ptx::umma_ss_pair(acc, ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B),
-                                ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B), idesc,
-                                (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::kSwizzle128B);
+            const uint64_t db = ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::kSwizzle128B);
+            if (!issuer) continue;
+            if constexpr (F8) ptx::umma_ss_pair_f8(acc, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            else ptx::umma_ss_pair(acc, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
           if (issuer) ptx::umma_commit_pair(ptx::smem_u32(&empty[s]));
           issued = true;
         }

@@ -142,13 +142,13 @@ int dit_linear_fp8(const void* x8, const void* w8, const void* bias, void* out, 
                    const void* alpha, int64_t rows_per_group, float x_scale, float w_scale,
                    void* stream);
 
-/* Kernel form of the bf16 dit_linear for later calls in this process: 1 (default) runs
- * CTA pairs (cta_group::2) on 256 x 256 tiles, each SM loading half of every B tile, both
- * CTAs' loads completing on the even CTA's barrier; 0 one CTA per 128 x 256 tile. The two
- * give the same bits; measured on B200 at the 480P projection shapes the pair form is
- * 8-15 % faster. dit_linear_fp8 always runs the single-CTA form. No counterpart in the
- * source pages. A plain process-wide setting, not synchronised: set it before other
- * threads issue calls. Errors: DIT_ERR_SHAPE for any other value. */
+/* Kernel form of dit_linear and dit_linear_fp8 for later calls in this process: 1
+ * (default) runs CTA pairs (cta_group::2) on 256 x 256 tiles, each SM loading half of
+ * every B tile, both CTAs' loads completing on the even CTA's barrier; 0 one CTA per
+ * 128 x 256 tile. The two give the same bits; measured on B200 at the 480P projection
+ * shapes the pair form is 8-15 % faster in bf16. No counterpart in the source pages. A
+ * plain process-wide setting, not synchronised: set it before other threads issue
+ * calls. Errors: DIT_ERR_SHAPE for any other value. */
 int dit_set_linear_variant(int variant);
 
 /* Standalone 3D-RoPE of q and k (DiT page, "3D-RoPE e atencao espaco-temporal"),

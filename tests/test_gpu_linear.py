@@ -130,7 +130,7 @@ def test_linear_wait_that_runs_out_reports_timeout():
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 208), (1000, 1024, 512), (77, 3072, 144)])
 @pytest.mark.parametrize("mode", ["plain", "bias_gelu", "gated"])
-def test_linear_fp8_parity(M, N, K, mode):
+def test_linear_fp8_parity(variant, M, N, K, mode):
     x, w = bits((M, K)), bits((N, K), std=K ** -0.5)
     inv_x, inv_w = 16.0, 256.0
     x8 = dit3d.dit_quantize_e4m3(to_dev(x), inv_x)
@@ -150,6 +150,22 @@ def test_linear_fp8_parity(M, N, K, mode):
     wd = oracle.quantize_e4m3(f64(w), inv_w) / inv_w
     ref = oracle.linear(xd, wd, **ref_kw)
     check_modulation(from_dev(out), ref, f"linear fp8 {mode} {M}x{N}x{K}")
+
+
+def test_linear_fp8_variants_agree():
+    M, N, K = 700, 1280, 960
+    x8 = dit3d.dit_quantize_e4m3(to_dev(bits((M, K))), 16.0)
+    w8 = dit3d.dit_quantize_e4m3(to_dev(bits((N, K), std=K ** -0.5)), 256.0)
+    outs = []
+    try:
+        for v in (0, 1):
+            dit3d.dit_set_linear_variant(v)
+            outs.append(dit3d.dit_linear_fp8(x8, w8, 1 / 16, 1 / 256))
+    finally:
+        dit3d.dit_set_linear_variant(DEFAULT_VARIANT)
+    dit3d.dit_check_device()
+    diff = (outs[0].float() - outs[1].float()).abs()
+    assert (diff <= outs[0].float().abs() * 2 ** -7 + 1e-6).all()
 
 
 def test_linear_fp8_errors():
