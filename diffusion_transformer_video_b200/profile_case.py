@@ -22,7 +22,7 @@ from . import dit3d
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", required=True,
-                    choices=["modulate", "residual", "rope", "attn", "euler", "linear"])
+                    choices=["modulate", "residual", "rope", "attn", "attn_rope", "euler", "linear"])
     ap.add_argument("--rows", type=int, required=True)
     ap.add_argument("--d-model", type=int, default=0, help="activation width (modulate, residual, euler)")
     ap.add_argument("--heads", type=int, default=0)
@@ -50,7 +50,7 @@ def main():
         call = {"modulate": lambda: dit3d.dit_adaln_modulate(x, prm[0], prm[1], rpg, out=out),
                 "residual": lambda: dit3d.dit_gated_residual(x, y, prm[0], rpg, out=out),
                 "euler": lambda: dit3d.dit_flow_euler_step(x, y, dt, rpg, out=out)}[a.kernel]
-    elif a.kernel in ("rope", "attn"):
+    elif a.kernel in ("rope", "attn", "attn_rope"):
         H, d = a.heads, a.head_dim
         q, k, v = bf(rows, H, d), bf(rows, H, d), bf(rows, H, d)
         frame = a.grid[0] * a.grid[1]
@@ -62,7 +62,9 @@ def main():
             call = lambda: dit3d.dit_rope3d_qk(q, k, desc, q_out=qo, k_out=ko)
         else:
             o = torch.empty_like(q)
-            call = lambda: dit3d.dit_attn_fwd(q, k, v, out=o)
+            # attn_rope: q and k rotated inside the attention kernel (fused 3D-RoPE)
+            rope = desc if a.kernel == "attn_rope" else None
+            call = lambda: dit3d.dit_attn_fwd(q, k, v, out=o, rope=rope)
     else:
         K, N = D, a.n_out or 3 * D
         x, w = bf(rows, K), bf(N, K, std=K ** -0.5)
