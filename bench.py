@@ -40,11 +40,11 @@ METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB2
 UNIT = "TFLOP/s"
 # DRAM bytes per head of one attention launch at the 480P geometry, from an ncu capture
 # with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum = 406.48 + 117.93 MB, over
-# 16), keyed by RoPE mode ("prepass" and "none" run the same kernel, without in-kernel
-# RoPE). Heads are independent, so a launch's traffic is this times its head count.
-# None where the current kernel has not been captured; other workloads report null.
+# 16; with in-kernel RoPE 407.39 + 119.45 MB), keyed by RoPE mode ("prepass" and "none"
+# run the same kernel, without in-kernel RoPE). Heads are independent, so a launch's
+# traffic is this times its head count. Other workloads report null.
 ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 524.411392e6 / 16, "none": 524.411392e6 / 16,
-                                 "fused": None}
+                                 "fused": 526.841856e6 / 16}
 
 
 def _peaks():
