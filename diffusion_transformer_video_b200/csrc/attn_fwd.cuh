@@ -16,7 +16,8 @@
 //   WG2 (warps 8-11) 3D-RoPE: rotate Q0/Q1 and every K_j in shared memory, in
 //                    place, right after TMA lands them (fp32 math, bf16 result).
 //   warp 12          TMA producer of Q0, Q1 (once) and of the 2-stage K ring.
-//   warp 13          TMEM allocator and tcgen05.mma issuer (one thread).
+//   warp 13          TMEM allocator and tcgen05.mma issuer (the whole warp runs the
+//                    loop, one elected lane issues).
 //   warp 14          TMA producer of the 2-stage V ring.
 //   warp 15          idle (it only gives its registers away).
 // A K stage is released right after both QK^T products read it, a V stage after
@@ -29,9 +30,9 @@
 // S_i once the softmax has read S_i into registers.
 // MMA order (ping-pong, so one tile's softmax overlaps the other tile's MMAs):
 //   S0=Q0K0, S1=Q1K0, then for each j: O0+=P0V_j, S0=Q0K_{j+1}, O1+=P1V_j, S1=Q1K_{j+1}.
-// Tensor-core operations issued by one thread run in order, and a commit arrives
-// only when every earlier operation of that thread is complete, so when the
-// softmax sees S_i(j+1) the product O_i += P_i(j)V_j has landed and O_i may be
+// Tensor-core operations issued by one thread (the elected lane) run in order, and a
+// commit arrives only when every earlier operation of that thread is complete, so when
+// the softmax sees S_i(j+1) the product O_i += P_i(j)V_j has landed and O_i may be
 // rescaled in place.
 // Online softmax in base 2 with a lazily updated row maximum: the running max is
 // only raised (and O, l rescaled) when a new score exceeds it by more than 2^8,

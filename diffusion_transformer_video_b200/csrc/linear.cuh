@@ -16,8 +16,9 @@
 // L2). 256 threads:
 //   warp 0     TMA producer: A (128 x 64) and B (256 x 64) boxes with the 128-byte
 //              swizzle into a 4-stage ring (48 KB per stage)
-//   warp 1     TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma
-//              M128 N256 K16 per stage into one of two 256-column accumulators
+//   warp 1     TMEM allocator and MMA issuer (whole warp, one elected lane):
+//              4 x tcgen05.mma M128 N256 K16 per stage into one of two 256-column
+//              accumulators
 //   warps 4-7  epilogue: thread = output row = TMEM lane; tcgen05.ld 32 columns at a
 //              time, bias / GELU / gate in fp32, one bf16 rounding, 16-byte stores
 // The two accumulators let the epilogue of tile i overlap the main loop of tile i+1.
