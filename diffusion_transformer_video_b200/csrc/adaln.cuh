@@ -16,6 +16,19 @@ namespace dit3d {
 
 constexpr int kRowThreads = 128;
 
+// Sum over a block of WARPS warps (warp shuffles, then one shared-memory exchange).
+template <int WARPS>
+__device__ __forceinline__ float block_sum_w(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = v;
+  __syncthreads();
+  float t = red[0];
+#pragma unroll
+  for (int w = 1; w < WARPS; ++w) t += red[w];
+  return t;
+}
 __device__ __forceinline__ float block_sum_128(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -30,12 +43,16 @@ __device__ __forceinline__ float block_sum_128(float v, float* red) {
 // parameter group per frame (1560 rows) the early form moves 5.3 TB/s against 4.3;
 // with a few large groups (a group per sample) the late form is faster (5.5 against
 // 5.2 TB/s), its parameter reads hitting in L1.
-template <int NV, bool EARLY>
-__global__ void __launch_bounds__(kRowThreads)
+// TH threads per row (TH / 32 warps). The launch uses 64 for the late form at
+// d_model <= 3072: the row's registers then limit an SM to 14 resident rows instead of
+// 10 with 128 threads, measured +10 % inside the 720P step (4.99 against 4.49 TB/s);
+// the early form keeps 128 (with 64 its 119 registers would leave 8 rows per SM).
+template <int NV, bool EARLY, int TH = kRowThreads>
+__global__ void __launch_bounds__(TH)
 adaln_modulate_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ gamma,
                       const __nv_bfloat16* __restrict__ beta, __nv_bfloat16* out, int32_t D,
                       int64_t rows_per_group, float eps, float scale_offset) {
-  __shared__ float red[2][4];
+  __shared__ float red[2][TH / 32];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const int nchunk = D >> 3;
@@ -46,7 +63,7 @@ adaln_modulate_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ 
   uint4 v[NV], gv_e[EARLY ? NV : 1], bv_e[EARLY ? NV : 1];
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
-    const int c = tid + k * kRowThreads;
+    const int c = tid + k * TH;
     v[k] = (c < nchunk) ? ld_stream(xr + c * 16) : make_uint4(0, 0, 0, 0);
     if constexpr (EARLY) {
       if (c < nchunk) {
@@ -62,11 +79,11 @@ adaln_modulate_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ 
 #pragma unroll
     for (int e = 0; e < 4; ++e) s += bf16lo(w[e]) + bf16hi(w[e]);
   }
-  const float mean = block_sum_128(s, red[0]) / static_cast<float>(D);
+  const float mean = block_sum_w<TH / 32>(s, red[0]) / static_cast<float>(D);
   float q = 0.f;
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
-    if (tid + k * kRowThreads < nchunk) {
+    if (tid + k * TH < nchunk) {
       const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -76,12 +93,12 @@ adaln_modulate_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ 
       }
     }
   }
-  const float var = block_sum_128(q, red[1]) / static_cast<float>(D);
+  const float var = block_sum_w<TH / 32>(q, red[1]) / static_cast<float>(D);
   const float rstd = rsqrtf(var + eps);
   char* orow = reinterpret_cast<char*>(out) + row * static_cast<int64_t>(D) * 2;
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
-    const int c = tid + k * kRowThreads;
+    const int c = tid + k * TH;
     if (c < nchunk) {
       uint4 gv, bv;
       if constexpr (EARLY) {

@@ -2,6 +2,7 @@
 // maps, the RoPE cos/sin table cache and kernel launches. All device work is in
 // the kernels of adaln.cuh, rope3d.cuh and attn_fwd.cuh.
 #include <algorithm>
+#include <type_traits>
 #include <chrono>
 #include <cmath>
 #include <cstdint>
@@ -323,6 +324,24 @@ constexpr int64_t kEarlyParamRows = 8192;
 template <int NV>
 void launch_modulate(const void* x, const void* g, const void* b, void* o, int64_t rows, int32_t D,
                      int64_t rpg, float eps, float s0, cudaStream_t st) {
+  // late form at d_model <= 3072: 64 threads per row, NV64 = ceil(D / 512) chunks each
+  if (rpg >= kEarlyParamRows && D <= 3072) {
+    const int nv64 = (D + 511) / 512;
+    auto run = [&](auto nv_tag) {
+      constexpr int NV64 = decltype(nv_tag)::value;
+      adaln_modulate_kernel<NV64, false, 64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
+          static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
+    };
+    switch (nv64) {
+      case 1: run(std::integral_constant<int, 1>{}); return;
+      case 2: run(std::integral_constant<int, 2>{}); return;
+      case 3: run(std::integral_constant<int, 3>{}); return;
+      case 4: run(std::integral_constant<int, 4>{}); return;
+      case 5: run(std::integral_constant<int, 5>{}); return;
+      default: run(std::integral_constant<int, 6>{}); return;
+    }
+  }
   if (rpg < kEarlyParamRows) {
     adaln_modulate_kernel<NV, true><<<static_cast<unsigned>(rows), kRowThreads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
