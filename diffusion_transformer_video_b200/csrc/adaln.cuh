@@ -45,8 +45,9 @@ __device__ __forceinline__ float block_sum_128(float v, float* red) {
 // 5.2 TB/s), its parameter reads hitting in L1.
 // TH threads per row (TH / 32 warps). The launch uses 64 for the late form at
 // d_model <= 3072: the row's registers then limit an SM to 14 resident rows instead of
-// 10 with 128 threads, measured +10 % inside the 720P step (4.99 against 4.49 TB/s);
-// the early form keeps 128 (with 64 its 119 registers would leave 8 rows per SM).
+// 10 with 128 threads, measured +10 % inside the 720P step (4.99 against 4.49 TB/s).
+// At d_model <= 3072 the early form is replaced by adaln_modulate_staged_kernel (with
+// 64 threads its 119 registers would leave 8 rows per SM).
 template <int NV, bool EARLY, int TH = kRowThreads>
 __global__ void __launch_bounds__(TH)
 adaln_modulate_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ gamma,
@@ -108,6 +109,84 @@ adaln_modulate_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ 
         gv = ld_cached(gr + c * 16);
         bv = ld_cached(br + c * 16);
       }
+      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lo = fmaf((bf16lo(w[e]) - mean) * rstd, scale_offset + bf16lo(gw[e]), bf16lo(bw[e]));
+        const float hi = fmaf((bf16hi(w[e]) - mean) * rstd, scale_offset + bf16hi(gw[e]), bf16hi(bw[e]));
+        o[e] = pack_bf16x2(lo, hi);
+      }
+      st_stream(orow + c * 16, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+}
+
+// The early form with the parameters staged in shared memory instead of registers:
+// gamma and beta are copied with cp.async (L1-allocating) when x is loaded, each thread
+// reading back only its own chunks after its own copies completed, so the row needs the
+// late form's registers (14 resident rows of 64 threads per SM at d_model 3072, against
+// 8 rows for the register-held early form). Measured on B200 inside the packed-varlen
+// step (one parameter group per frame): 5.06-5.10 against 4.71-4.75 TB/s; with the
+// L2-only copy (cp.async.cg) it was twice as slow, every row then refetching its
+// parameters from L2.
+template <int NV, int TH>
+__global__ void __launch_bounds__(TH)
+adaln_modulate_staged_kernel(const __nv_bfloat16* x, const __nv_bfloat16* __restrict__ gamma,
+                             const __nv_bfloat16* __restrict__ beta, __nv_bfloat16* out, int32_t D,
+                             int64_t rows_per_group, float eps, float scale_offset) {
+  __shared__ float red[2][TH / 32];
+  __shared__ uint4 gb[2 * NV * TH];  // [gamma chunks | beta chunks], chunk k of thread t at k * TH + t
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int nchunk = D >> 3;
+  const char* xr = reinterpret_cast<const char*>(x) + row * static_cast<int64_t>(D) * 2;
+  const int64_t g = row / rows_per_group;
+  const char* gr = reinterpret_cast<const char*>(gamma) + g * static_cast<int64_t>(D) * 2;
+  const char* br = reinterpret_cast<const char*>(beta) + g * static_cast<int64_t>(D) * 2;
+  uint4 v[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int c = tid + k * TH;
+    v[k] = (c < nchunk) ? ld_stream(xr + c * 16) : make_uint4(0, 0, 0, 0);
+    if (c < nchunk) {
+      cp_async16(&gb[k * TH + tid], gr + c * 16);
+      cp_async16(&gb[(NV + k) * TH + tid], br + c * 16);
+    }
+  }
+  cp_async_commit();
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s += bf16lo(w[e]) + bf16hi(w[e]);
+  }
+  const float mean = block_sum_w<TH / 32>(s, red[0]) / static_cast<float>(D);
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    if (tid + k * TH < nchunk) {
+      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = bf16lo(w[e]) - mean, b = bf16hi(w[e]) - mean;
+        q = fmaf(a, a, q);
+        q = fmaf(b, b, q);
+      }
+    }
+  }
+  const float var = block_sum_w<TH / 32>(q, red[1]) / static_cast<float>(D);
+  const float rstd = rsqrtf(var + eps);
+  cp_async_wait_all();
+  char* orow = reinterpret_cast<char*>(out) + row * static_cast<int64_t>(D) * 2;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int c = tid + k * TH;
+    if (c < nchunk) {
+      const uint4 gv = gb[k * TH + tid], bv = gb[(NV + k) * TH + tid];
       const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
       const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};

@@ -62,5 +62,13 @@ __device__ __forceinline__ uint4 ld_cached(const void* p) {
 __device__ __forceinline__ void st_stream(void* p, uint4 v) {
   __stcs(reinterpret_cast<uint4*>(p), v);
 }
+// 16-byte asynchronous copy global -> shared (L1-allocating), its group commit, and the
+// wait for all of the calling thread's committed copies.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 }  // namespace dit3d

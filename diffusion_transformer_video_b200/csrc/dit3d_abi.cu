@@ -324,14 +324,20 @@ constexpr int64_t kEarlyParamRows = 8192;
 template <int NV>
 void launch_modulate(const void* x, const void* g, const void* b, void* o, int64_t rows, int32_t D,
                      int64_t rpg, float eps, float s0, cudaStream_t st) {
-  // late form at d_model <= 3072: 64 threads per row, NV64 = ceil(D / 512) chunks each
-  if (rpg >= kEarlyParamRows && D <= 3072) {
+  // d_model <= 3072: 64 threads per row, NV64 = ceil(D / 512) chunks each; large parameter
+  // groups take the late form, small ones the form with parameters staged in shared memory
+  if (D <= 3072) {
     const int nv64 = (D + 511) / 512;
     auto run = [&](auto nv_tag) {
       constexpr int NV64 = decltype(nv_tag)::value;
-      adaln_modulate_kernel<NV64, false, 64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
-          static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
+      if (rpg >= kEarlyParamRows)
+        adaln_modulate_kernel<NV64, false, 64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
+            static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
+      else
+        adaln_modulate_staged_kernel<NV64, 64><<<static_cast<unsigned>(rows), 64, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g),
+            static_cast<const __nv_bfloat16*>(b), static_cast<__nv_bfloat16*>(o), D, rpg, eps, s0);
     };
     switch (nv64) {
       case 1: run(std::integral_constant<int, 1>{}); return;
