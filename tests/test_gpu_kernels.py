@@ -31,9 +31,11 @@ def test_adaln_modulate_parity(rows, D, rpg, s0):
 
 
 @pytest.mark.parametrize("rows,D,rpg", [(9000, 3072, 1500), (4000, 5120, 400), (30000, 128, 1000),
-                                        (20000, 1032, 20)])
+                                        (20000, 1032, 20), (16384, 1032, 16384), (10000, 2048, 10000)])
 def test_adaln_modulate_large_and_in_place(rows, D, rpg):
-    # many rows and groups (ragged widths included), out of place and in place over x
+    # many rows and groups (ragged widths included), out of place and in place over x; groups
+    # of 8192 rows or more take the late form (64 threads per row up to d_model 3072), shorter
+    # ones the form with gamma / beta staged in shared memory
     x, g, b = bits((rows, D)), bits((rows // rpg, D), 0.1), bits((rows // rpg, D), 0.1)
     xt = to_dev(x)
     out = dit3d.dit_adaln_modulate(xt, to_dev(g), to_dev(b), rpg)
