@@ -4,8 +4,8 @@
 //   x' = x + alpha * SelfAttn(gamma * LN(x) + beta); alpha starts at zero so the
 //   block is the identity.
 //
-// One CTA of kRowThreads threads owns one token row. Each thread keeps its NV
-// 16-byte chunks of the row in registers, so x is read from HBM exactly once and
+// One CTA of kRowThreads threads (64 for the modulation at d_model <= 3072) owns one
+// token row. Each thread keeps its NV 16-byte chunks of the row in registers, so x is read from HBM exactly once and
 // the output written once (4 bytes of traffic per element for the modulation,
 // 6 for the residual). Mean and variance are two warp-shuffle + shared-memory
 // reductions over the register-resident row (variance around the mean, fp32).
