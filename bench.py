@@ -572,9 +572,34 @@ def main():
         dit3d.dit_check_device()
         t_q8 = statistics.mean(e[0].elapsed_time(e[1]) for e in ev3)
         t_a8 = statistics.mean(e[1].elapsed_time(e[2]) for e in ev3)
+        # the E4M3 operands straight from the unrotated q, k: RoPE and quantisation in
+        # one pass, against the bf16 RoPE pass followed by the two quantisations
+        q8f = torch.empty_like(q8)
+        k8f = torch.empty_like(k8)
+
+        def rope_e4m3():
+            dit3d.dit_rope3d_qk_e4m3(dev["q"], dev["k"], run.desc, 64.0, 64.0, n_seq=w.n_seq,
+                                     cu_seqlens=cu, q8_out=q8f, k8_out=k8f)
+        for _ in range(3):
+            rope_e4m3()
+        ev5 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(max(K, 3))]
+        for a, b in ev5:
+            a.record(stream)
+            rope_e4m3()
+            b.record(stream)
+        torch.cuda.synchronize()
+        dit3d.dit_check_device()
+        t_rq8 = statistics.mean(a.elapsed_time(b) for a, b in ev5)
+        rq8_bytes = 3.0 * rows * H * d * 2  # bf16 q, k read; E4M3 q, k written
         fp8 = {"ms": t_a8, "TFLOP/s": w.attn_flops() / (t_a8 * 1e-3) / 1e12,
                "quantize_ms": t_q8, "max_abs_vs_bf16_attention": float((o8.float() - o.float()).abs().max()),
+               "rope_e4m3": {"ms": t_rq8, "GB/s": rq8_bytes / (t_rq8 * 1e-3) / 1e9,
+                             "two_pass_ms": t["rope"] + t_q8,
+                             "bytes_equal_two_pass": bool(torch.equal(q8f, q8) and torch.equal(k8f, k8)),
+                             "kernel": "dit_rope3d_qk_e4m3 (RoPE and E4M3 in one pass)"},
                "in_step": False, "note": "E4M3 q, k (scale 1/64), bf16 P and V"}
+        del q8f, k8f
         # all of q, k, v (and P) in E4M3
         v8 = dit3d.dit_quantize_e4m3(dev["v"], 64.0)
         for _ in range(2):

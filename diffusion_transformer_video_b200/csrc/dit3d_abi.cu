@@ -639,13 +639,41 @@ int dit_set_linear_variant(int variant) {
   return DIT_OK;
 }
 
-int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,
-                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
-                  const int32_t* cu_seqlens_host, const dit_rope3d_desc* rope, void* stream) {
+}  // extern "C"
+
+namespace {
+// [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void* a, int64_t na, const void* b, int64_t nb) {
+  const auto pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + static_cast<uintptr_t>(nb) && pb < pa + static_cast<uintptr_t>(na);
+}
+
+// Shared body of dit_rope3d_qk (bf16 out) and dit_rope3d_qk_e4m3 (E4M3 codes out).
+int rope3d_qk_impl(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,
+                   int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                   const int32_t* cu_seqlens_host, const dit_rope3d_desc* rope, bool e4m3,
+                   float q_inv, float k_inv, void* stream) {
   if (!q_in || !q_out || !rope || (k_in && !k_out)) return DIT_ERR_NULL;
   if (rows < 0 || H <= 0 || (d != 64 && d != 128)) return DIT_ERR_SHAPE;
-  if (!aligned16(q_in) || !aligned16(q_out) || (k_in && (!aligned16(k_in) || !aligned16(k_out))))
+  if (e4m3 && (!std::isfinite(q_inv) || (k_in && !std::isfinite(k_inv)))) return DIT_ERR_SHAPE;
+  if (!aligned16(q_in) || !aligned16(k_in)) return DIT_ERR_ALIGN;
+  const uintptr_t out_mask = e4m3 ? 7u : 15u;
+  if ((reinterpret_cast<uintptr_t>(q_out) & out_mask) ||
+      (k_in && (reinterpret_cast<uintptr_t>(k_out) & out_mask)))
     return DIT_ERR_ALIGN;
+  if (e4m3) {
+    // codes are half the size of their sources: a chunk written by one thread could
+    // land on a source chunk another thread has yet to read
+    const int64_t n = rows * H * d;
+    const void* ins[2] = {q_in, k_in};
+    void* outs[2] = {q_out, k_in ? k_out : nullptr};
+    for (void* o : outs) {
+      if (!o) continue;
+      for (const void* i : ins)
+        if (i && overlaps(o, n, i, 2 * n)) return DIT_ERR_SHAPE;
+    }
+    if (outs[1] && overlaps(outs[0], n, outs[1], n)) return DIT_ERR_SHAPE;
+  }
   std::vector<int64_t> lens;
   if (int s = check_seqs(rows, n_seq, cu_seqlens_dev, cu_seqlens_host, &lens)) return s;
   int t_ext = 0;
@@ -657,15 +685,39 @@ int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, 
   if (int s = get_table(rope, t_ext, st, &rp)) return s;
   const int64_t dense_len = cu_seqlens_dev ? 0 : rows / n_seq;
   const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
-  if (d == 128)
-    rope3d_qk_kernel<128><<<grid, 256, 0, st>>>(
-        static_cast<const uint4*>(q_in), static_cast<const uint4*>(k_in), static_cast<uint4*>(q_out),
-        static_cast<uint4*>(k_out), rows, H, cu_seqlens_dev, n_seq, dense_len, rp);
-  else
-    rope3d_qk_kernel<64><<<grid, 256, 0, st>>>(
-        static_cast<const uint4*>(q_in), static_cast<const uint4*>(k_in), static_cast<uint4*>(q_out),
-        static_cast<uint4*>(k_out), rows, H, cu_seqlens_dev, n_seq, dense_len, rp);
+  const auto* qi = static_cast<const uint4*>(q_in);
+  const auto* ki = static_cast<const uint4*>(k_in);
+  auto launch = [&](auto d_head, auto quant) {
+    rope3d_qk_kernel<decltype(d_head)::value, decltype(quant)::value><<<grid, 256, 0, st>>>(
+        qi, ki, q_out, k_out, rows, H, cu_seqlens_dev, n_seq, dense_len, rp, q_inv, k_inv);
+  };
+  using D128 = std::integral_constant<int, 128>;
+  using D64 = std::integral_constant<int, 64>;
+  if (e4m3) {
+    if (d == 128) launch(D128{}, std::true_type{}); else launch(D64{}, std::true_type{});
+  } else {
+    if (d == 128) launch(D128{}, std::false_type{}); else launch(D64{}, std::false_type{});
+  }
   return launch_status();
+}
+}  // namespace
+
+extern "C" {
+
+int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,
+                  int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
+                  const int32_t* cu_seqlens_host, const dit_rope3d_desc* rope, void* stream) {
+  return rope3d_qk_impl(q_in, k_in, q_out, k_out, rows, H, d, n_seq, cu_seqlens_dev,
+                        cu_seqlens_host, rope, false, 1.f, 1.f, stream);
+}
+
+int dit_rope3d_qk_e4m3(const void* q_in, const void* k_in, void* q8_out, void* k8_out,
+                       int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                       const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                       const dit_rope3d_desc* rope, float q_inv_scale, float k_inv_scale,
+                       void* stream) {
+  return rope3d_qk_impl(q_in, k_in, q8_out, k8_out, rows, H, d, n_seq, cu_seqlens_dev,
+                        cu_seqlens_host, rope, true, q_inv_scale, k_inv_scale, stream);
 }
 
 int dit_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t rows,

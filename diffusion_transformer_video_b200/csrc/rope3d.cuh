@@ -22,6 +22,7 @@
 // The position offsets are folded into the angles.
 #pragma once
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace dit3d {
 
@@ -171,11 +172,16 @@ __device__ __forceinline__ uint4 rope_chunk_reg(uint4 v, int nb, const float4 (&
 // storing them. Same per-chunk arithmetic as rope_chunk (and the attention kernel),
 // so all produce the same bits. In place (q_out == q_in) is safe: every element is
 // read and written by the same thread.
-template <int D_HEAD>
-__global__ void __launch_bounds__(256)
-rope3d_qk_kernel(const uint4* q_in, const uint4* k_in, uint4* q_out, uint4* k_out, int64_t rows,
+// With E4M3 set the rotated chunk, rounded to bf16 as above, is scaled by q_inv (k_inv)
+// and written as 8 E4M3 codes (8 bytes) with quantize_e4m3_kernel's conversion: the
+// same bytes as the rotation followed by the separate quantisation pass, without
+// writing and re-reading the rotated bf16 tensors. The outputs then hold half the
+// bytes of the inputs, so they must not overlap them.
+template <int D_HEAD, bool E4M3 = false>
+__global__ void __launch_bounds__(256, 3)
+rope3d_qk_kernel(const uint4* q_in, const uint4* k_in, void* q_out, void* k_out, int64_t rows,
                  int32_t H, const int32_t* __restrict__ cu, int32_t n_seq, int64_t dense_len,
-                 RopeParams rp) {
+                 RopeParams rp, float q_inv = 1.f, float k_inv = 1.f) {
   constexpr int kCpr = D_HEAD / 8;  // 16-byte chunks per head
   constexpr int kUnroll = 4;
   static_assert(32 % kCpr == 0, "lane-fixed chunks need D_HEAD/8 to divide 32");
@@ -222,8 +228,20 @@ rope3d_qk_kernel(const uint4* q_in, const uint4* k_in, uint4* q_out, uint4* k_ou
     for (int u = 0; u < kUnroll; ++u) {
       const int c = c0 + 32 * u;
       if (c < nchunk) {
-        q_out[base + c] = rope_chunk_reg(vq[u], nb, f);
-        if (has_k) k_out[base + c] = rope_chunk_reg(vk[u], nb, f);
+        const uint4 rq = rope_chunk_reg(vq[u], nb, f);
+        if constexpr (E4M3)
+          static_cast<uint2*>(q_out)[base + c] =
+              make_uint2(e4m3x4(rq.x, rq.y, q_inv), e4m3x4(rq.z, rq.w, q_inv));
+        else
+          static_cast<uint4*>(q_out)[base + c] = rq;
+        if (has_k) {
+          const uint4 rk = rope_chunk_reg(vk[u], nb, f);
+          if constexpr (E4M3)
+            static_cast<uint2*>(k_out)[base + c] =
+                make_uint2(e4m3x4(rk.x, rk.y, k_inv), e4m3x4(rk.z, rk.w, k_inv));
+          else
+            static_cast<uint4*>(k_out)[base + c] = rk;
+        }
       }
     }
   }

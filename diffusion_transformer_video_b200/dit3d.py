@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "DIT_OK", 1: "DIT_ERR_NULL", 2: "DIT_ERR_SHAPE", 3: "DIT_ERR_
 EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "dit_linear",
            "dit_linear_fp8",
            "dit_set_linear_variant", "dit_attn_fwd_qk8", "dit_attn_fwd_fp8", "dit_quantize_e4m3",
-           "dit_rope3d_qk", "dit_attn_fwd",
+           "dit_rope3d_qk", "dit_rope3d_qk_e4m3", "dit_attn_fwd",
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout",
            "dit_debug_wait_limit_ns", "dit_wait_device", "dit_debug_poll_fake", "dit_debug_exp2_fma")
@@ -71,6 +71,8 @@ def lib():
         L.dit_attn_fwd_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32, f32, f32, f32, P]
         L.dit_rope3d_qk.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
                                     ctypes.POINTER(RopeDesc), P]
+        L.dit_rope3d_qk_e4m3.argtypes = [P, P, P, P, i64, i32, i32, i32, P, P,
+                                         ctypes.POINTER(RopeDesc), f32, f32, P]
         L.dit_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
                                    ctypes.POINTER(RopeDesc), P]
         L.dit_attn_fwd_noalloc.argtypes = [P, P, P, P, P, i64, i32, i32, i32, P, P, f32,
@@ -270,6 +272,29 @@ def dit_attn_fwd(q, k, v, n_seq=1, cu_seqlens=None, rope: RopeDesc | None = None
 def _u8(t: torch.Tensor, name: str):
     if not (isinstance(t, torch.Tensor) and t.dtype == torch.uint8 and t.is_cuda and t.is_contiguous()):
         raise TypeError(f"{name} must be a contiguous uint8 (E4M3 codes) CUDA tensor")
+
+
+def dit_rope3d_qk_e4m3(q, k, rope: RopeDesc, q_inv_scale: float, k_inv_scale: float = 1.0,
+                       n_seq=1, cu_seqlens=None, q8_out=None, k8_out=None):
+    """3D-RoPE of q and k ([rows, H, d] bf16) written as E4M3 codes of the rotated
+    values times q_inv_scale / k_inv_scale. Returns (q8, k8) as uint8 tensors."""
+    _bf16(q, "q")
+    if k is not None:
+        _bf16(k, "k")
+    q8_out = torch.empty(q.shape, dtype=torch.uint8, device=q.device) if q8_out is None else q8_out
+    _u8(q8_out, "q8_out")
+    if k is not None:
+        k8_out = (torch.empty(k.shape, dtype=torch.uint8, device=k.device) if k8_out is None
+                  else k8_out)
+        _u8(k8_out, "k8_out")
+    rows, H, d = q.shape
+    cu_dev, cu_host, ns = _cu_args(cu_seqlens)
+    n = ns if ns is not None else n_seq
+    _check(lib().dit_rope3d_qk_e4m3(_ptr(q), _ptr(k), _ptr(q8_out), _ptr(k8_out), rows, H, d, n,
+                                    _ptr(cu_dev), _ptr(cu_host), ctypes.byref(rope),
+                                    float(q_inv_scale), float(k_inv_scale), _stream()))
+    _keep(cu_dev)
+    return q8_out, k8_out
 
 
 def dit_quantize_e4m3(x, inv_scale: float, out=None):

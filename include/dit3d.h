@@ -10,6 +10,7 @@
  *   out = res + alpha_g * act(x w^T + b)  (projections, MLP)     dit_linear
  *   o   = attention on E4M3 q, k (and v, P)                     dit_attn_fwd_qk8 / _fp8
  *   q8  = e4m3(x * inv_scale)                                   dit_quantize_e4m3
+ *   q8,k8 = e4m3(R3D q * inv_q), e4m3(R3D k * inv_k)               dit_rope3d_qk_e4m3
  *
  * Formulas: "DiT, Flow Matching e 3D Attention: A Engenharia de Video com IA",
  * sections "A ruptura da U-Net" (adaLN-Zero) and "3D-RoPE e atencao
@@ -162,6 +163,25 @@ int dit_set_linear_variant(int variant);
 int dit_rope3d_qk(const void* q_in, const void* k_in, void* q_out, void* k_out, int64_t rows,
                   int32_t H, int32_t d, int32_t n_seq, const int32_t* cu_seqlens_dev,
                   const int32_t* cu_seqlens_host, const dit_rope3d_desc* rope, void* stream);
+
+/* dit_rope3d_qk followed by E4M3 quantisation of its outputs, in one pass (DiT page,
+ * "3D-RoPE e atencao espaco-temporal" for the rotation; "Engenharia de inferencia e
+ * paralelismo de contexto: Ulysses, Ring Attention e FP8" for the FP8 operands):
+ *   q8_out = e4m3(bf16(R3D q) * q_inv_scale),  k8_out = e4m3(bf16(R3D k) * k_inv_scale)
+ * byte for byte what dit_rope3d_qk into bf16 buffers followed by dit_quantize_e4m3
+ * of each gives, without writing and re-reading the rotated bf16 tensors: the
+ * operands of dit_attn_fwd_qk8 / dit_attn_fwd_fp8.
+ *   q_in, k_in     : [rows, H, d] bf16, 16-byte aligned; k_in may be NULL (k8_out
+ *                    and k_inv_scale are then ignored)
+ *   q8_out, k8_out : [rows, H, d] E4M3 codes, one byte each, 8-byte aligned; they
+ *                    must overlap neither input nor each other (no in-place form)
+ * Errors: as dit_rope3d_qk; DIT_ERR_SHAPE for an inverse scale that is not finite or
+ * for overlapping buffers; DIT_ERR_ALIGN for misaligned pointers. */
+int dit_rope3d_qk_e4m3(const void* q_in, const void* k_in, void* q8_out, void* k8_out,
+                       int64_t rows, int32_t H, int32_t d, int32_t n_seq,
+                       const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                       const dit_rope3d_desc* rope, float q_inv_scale, float k_inv_scale,
+                       void* stream);
 
 /* Full non-causal attention per sequence and head (DiT page, "3D-RoPE e atencao
  * espaco-temporal"; the Flowception summary: bidirectional attention over all

@@ -54,6 +54,11 @@ def test_guards_survive_every_kernel():
     dit3d.dit_rope3d_qk(q, k, desc, q_out=qo, k_out=ko)
     dit3d.dit_check_device()
     checks += [("rope q", _intact(qb, qo.numel())), ("rope k", _intact(kb, ko.numel()))]
+    q8b, q8o = _guarded((rows, H, d), torch.uint8)
+    k8b, k8o = _guarded((rows, H, d), torch.uint8)
+    dit3d.dit_rope3d_qk_e4m3(q, k, desc, 64.0, 32.0, q8_out=q8o, k8_out=k8o)
+    dit3d.dit_check_device()
+    checks += [("rope e4m3 q", _intact(q8b, q8o.numel())), ("rope e4m3 k", _intact(k8b, k8o.numel()))]
 
     mb, mo = _guarded((rows, D), torch.bfloat16)
     dit3d.dit_adaln_modulate(x, gamma, beta, 111, out=mo)

@@ -67,6 +67,67 @@ def test_attn_qk8_after_rope_pass():
     check_attention(from_dev(o), ref, "qk8 after rope")
 
 
+def _e4m3_step(v: np.ndarray) -> np.ndarray:
+    """Spacing of E4M3 values at |v| (3 mantissa bits; subnormal step 2^-9)."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -6)))
+    return np.ldexp(1.0, (e - 3).astype(np.int64))
+
+
+@pytest.mark.parametrize("d,bands,gh,gw,frames,H,q_inv,k_inv,with_k", [
+    (128, (44, 42, 42), 5, 6, [7, 3], 3, 64.0, 16.0, True),
+    (128, (44, 42, 42), 30, 52, [1], 40, 256.0, 256.0, True),  # the 480P row width
+    (64, (16, 24, 24), 4, 4, [2, 1, 3], 2, 1.0, 512.0, True),   # saturation at 448
+    (128, (6, 0, 122), 3, 4, [2, 3], 5, 64.0, 0.25, True),      # empty middle band
+    (64, (20, 44, 0), 3, 3, [2], 7, 8.0, 1.0, False),           # q only
+])
+def test_rope3d_e4m3_equals_rope_then_quantize(d, bands, gh, gw, frames, H, q_inv, k_inv, with_k):
+    lens = [f * gh * gw for f in frames]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    rows = int(cu[-1])
+    rng = np.random.default_rng(rows + H)
+    mk = lambda: wl.f32_to_bf16_bits(rng.standard_normal((rows, H, d)).astype(np.float32))
+    q, k = mk(), mk() if with_k else None
+    desc = dit3d.rope_desc(gh, gw, bands, 10000.0, (1, 0, 2))
+    qd, kd = to_dev(q), (to_dev(k) if with_k else None)
+    q8, k8 = dit3d.dit_rope3d_qk_e4m3(qd, kd, desc, q_inv, k_inv, cu_seqlens=cu)
+    qr, kr = dit3d.dit_rope3d_qk(qd, kd, desc, cu_seqlens=cu)
+    dit3d.dit_check_device()
+    # byte for byte the two-pass route
+    assert torch.equal(q8, dit3d.dit_quantize_e4m3(qr, q_inv))
+    if with_k:
+        assert torch.equal(k8, dit3d.dit_quantize_e4m3(kr, k_inv))
+    else:
+        assert k8 is None
+    # and the oracle's codes of its own rotation rounded to bf16: equal, except where
+    # the fp32 and fp64 rotations round to neighbouring bf16 values, one E4M3 step
+    for got, src, inv in ((q8, q, q_inv),) + (((k8, k, k_inv),) if with_k else ()):
+        rot = oracle.rope3d(f64(src), cu, gh, gw, bands, 10000.0, (1, 0, 2))
+        ref = oracle.quantize_e4m3(oracle.round_bf16(rot), inv)
+        dec = _decode(got)
+        diff = np.abs(dec - ref)
+        assert (diff <= _e4m3_step(np.maximum(np.abs(dec), np.abs(ref)))).all()
+        assert (diff == 0).mean() > 0.999
+
+
+def test_rope3d_e4m3_errors():
+    desc = dit3d.rope_desc(2, 2, (44, 42, 42))
+    q = torch.zeros(8, 1, 128, dtype=torch.bfloat16, device="cuda")
+    L = dit3d.lib()
+    import ctypes
+    args = lambda qi, ki, qo, ko, qs=1.0: (qi, ki, qo, ko, 8, 1, 128, 2, None, None,
+                                           ctypes.byref(desc), qs, 1.0, None)
+    qp = q.data_ptr()
+    # the codes may not overwrite their own (or the other) source
+    assert L.dit_rope3d_qk_e4m3(*args(qp, None, qp, None)) == 2
+    assert L.dit_rope3d_qk_e4m3(*args(qp, None, qp + 1024, None)) == 2
+    out = torch.empty(8, 1, 128, dtype=torch.uint8, device="cuda")
+    assert L.dit_rope3d_qk_e4m3(*args(qp, None, out.data_ptr() + 4, None)) == 3  # 8-byte alignment
+    assert L.dit_rope3d_qk_e4m3(*args(qp, None, out.data_ptr(), None, float("inf"))) == 2
+    assert L.dit_rope3d_qk_e4m3(*args(qp, None, None, None)) == 1
+    assert L.dit_rope3d_qk_e4m3(*args(qp, None, out.data_ptr(), None)) == 0
+    dit3d.dit_check_device()
+
+
 def test_attn_qk8_errors():
     v = torch.zeros(10, 1, 64, dtype=torch.bfloat16, device="cuda")
     c = torch.zeros(10, 1, 64, dtype=torch.uint8, device="cuda")
