@@ -77,6 +77,22 @@ def test_validation_before_any_device_work(L):
                            ctypes.byref(dit3d.rope_desc(2, 2, (15, 25, 24))), None) == 2
     assert L.dit_rope3d_qk(FAKE, None, FAKE, None, 18, 2, 64, 1, None, None,
                            ctypes.byref(dit3d.rope_desc(2, 2, (16, 24, 24))), None) == 2
+    # RoPE with E4M3 output: codes overlapping a source, codes not 8-byte aligned, a
+    # scale that is not finite (q [16, 2, 128] bf16 spans 8 KB from FAKE)
+    rope = ctypes.byref(dit3d.rope_desc(2, 2, (44, 42, 42)))
+    e4 = lambda qi, ki, qo, ko, qs=1.0, ks=1.0: L.dit_rope3d_qk_e4m3(
+        qi, ki, qo, ko, 16, 2, 128, 1, None, None, rope, qs, ks, None)
+    apart, apart2 = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    k_in = ctypes.c_void_p(0x40000)
+    assert e4(FAKE, None, FAKE, None) == 2
+    assert e4(FAKE, None, ctypes.c_void_p(0x10000 + 8192 - 8), None) == 2
+    assert e4(FAKE, k_in, apart, ctypes.c_void_p(0x40000 + 4096)) == 2   # k codes on k
+    assert e4(FAKE, k_in, apart, ctypes.c_void_p(0x20000 + 4088)) == 2   # codes on codes
+    assert e4(FAKE, None, ctypes.c_void_p(0x20004), None) == 3
+    assert e4(FAKE, None, apart, None, float("nan")) == 2
+    assert e4(FAKE, k_in, apart, apart2, 1.0, float("inf")) == 2
+    assert e4(FAKE, None, None, None) == 1
+    assert e4(FAKE, k_in, apart, None) == 1
 
 
 @pytest.mark.skipif(os.environ.get("CUDA_VISIBLE_DEVICES", None) is None and
@@ -86,6 +102,9 @@ def test_valid_call_without_gpu_reports_device_error(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.dit_adaln_modulate(FAKE, FAKE, FAKE, FAKE, 4, 64, 4, 1e-6, 1.0, None) == 5
+    assert L.dit_rope3d_qk_e4m3(FAKE, None, ctypes.c_void_p(0x20000), None, 16, 2, 128, 1,
+                                None, None, ctypes.byref(dit3d.rope_desc(2, 2, (44, 42, 42))),
+                                64.0, 1.0, None) == 5
 
 
 def test_watchdog_poll_loop_with_a_fake_query(L):
