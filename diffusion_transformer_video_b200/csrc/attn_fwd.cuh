@@ -81,8 +81,16 @@ struct Params {
   // grid (n_order > 0); otherwise a (pairs, heads) grid in cu_seqlens order
   int32_t n_order;
   int32_t seq_order[64];
+  // dense batches: work units (a pair of query tiles of one sequence and head) are
+  // numbered head-major from unit0. kv_split > 1: a 1-D grid of clusters of kv_split
+  // CTAs, one cluster per unit, CTA s of a cluster taking key tiles
+  // [s * nk / kv_split, (s + 1) * nk / kv_split) and the cluster merging the partial
+  // results through distributed shared memory (the launch's last partial wave)
+  int32_t kv_split;
+  int32_t unit0;
 };
 constexpr int kMaxOrder = 64;
+constexpr int kMaxSplit = 8;  // portable cluster size
 
 template <int D>
 struct Smem {
@@ -93,6 +101,12 @@ struct Smem {
   static constexpr uint32_t kTab = kV + kVStages * kTile;     // RoPE cos/sin table copy
   static constexpr uint32_t kTabBytes = 32 * 1024;
   static constexpr uint32_t kBytes = kTab + kTabBytes;
+  // key-range split: once every MMA has completed, the Q/K/V area holds the CTA's
+  // partial O (fp32 rows of D + 4 floats: a row shift of 16 bytes keeps a warp's row
+  // stores conflict-free) for its 2 * kTileM query rows, then (m, l) per row
+  static constexpr uint32_t kPartStride = (D + 4) * 4;
+  static constexpr uint32_t kPartMl = 2 * kTileM * kPartStride;
+  static_assert(kPartMl + 2 * kTileM * 8 <= kTab, "partial results fit in the Q/K/V area");
   // dynamic smem request: forces one CTA per SM (the CTA takes all 512 TMEM columns)
   static constexpr uint32_t kRequest = (kBytes + 1024 > 120 * 1024) ? kBytes + 1024 : 120 * 1024;
 };
@@ -272,6 +286,67 @@ __device__ __forceinline__ void rope_tile_global(uint8_t* tile, int64_t row0, in
   }
 }
 
+// Merge of a key-range split (Params::kv_split): CTA `split` of the cluster combines
+// rows [split * 256 / n_split, (split + 1) * 256 / n_split) of the unit's 256 query rows
+// from every CTA's partial (O_s, m_s, l_s), read from their shared memory:
+//   M = max_s m_s,  w_s = 2^(m_s - M),  o = sum_s w_s O_s / sum_s w_s l_s,
+// the same rescaling the online softmax applies between key tiles, in a fixed order
+// of s. Thread t (of the 256 softmax threads) takes 16-byte output chunks t, t + 256, ...
+template <int D>
+__device__ __forceinline__ void merge_split_rows(uint8_t* smem, const Params& p, int split,
+                                                 int n_split, int64_t q_row0, int64_t seq_len,
+                                                 int64_t seq_start, int head, int t) {
+  using L = Smem<D>;
+  constexpr int kCh = D / 8;  // 16-byte output chunks (8 bf16) per row
+  constexpr int kRows = 2 * kTileM;
+  const int g0 = split * kRows / n_split, g1 = (split + 1) * kRows / n_split;
+  const uint32_t part = ptx::smem_u32(smem);
+#pragma unroll 1
+  for (int idx = t; idx < (g1 - g0) * kCh; idx += kRows) {
+    const int g = g0 + idx / kCh, c = idx % kCh;
+    const int64_t row_in_seq = q_row0 + g;
+    if (row_in_seq >= seq_len) continue;
+    float mt[kMaxSplit], lt[kMaxSplit];
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) {
+      if (s < n_split) {
+        const float2 v = ptx::ld_cluster_f2(ptx::mapa_shared(part + L::kPartMl + g * 8, s));
+        mt[s] = v.x;
+        lt[s] = v.y;
+        M = fmaxf(M, v.x);
+      }
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float lsum = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) {
+      if (s < n_split) {
+        const float w = ex2(mt[s] - M);
+        lsum = fmaf(w, lt[s], lsum);
+        const uint32_t a = ptx::mapa_shared(part + g * L::kPartStride + c * 32, s);
+        const float4 u0 = ptx::ld_cluster_f4(a), u1 = ptx::ld_cluster_f4(a + 16);
+        acc[0] = fmaf(w, u0.x, acc[0]);
+        acc[1] = fmaf(w, u0.y, acc[1]);
+        acc[2] = fmaf(w, u0.z, acc[2]);
+        acc[3] = fmaf(w, u0.w, acc[3]);
+        acc[4] = fmaf(w, u1.x, acc[4]);
+        acc[5] = fmaf(w, u1.y, acc[5]);
+        acc[6] = fmaf(w, u1.z, acc[6]);
+        acc[7] = fmaf(w, u1.w, acc[7]);
+      }
+    }
+    const float inv = p.o_scale / lsum;
+    uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
+                    ((seq_start + row_in_seq) * p.H + head) * static_cast<int64_t>(D) * 2;
+    *reinterpret_cast<uint4*>(orow + c * 16) =
+        make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                   pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+    if (c == 0 && p.lse != nullptr)
+      p.lse[(seq_start + row_in_seq) * p.H + head] = (M + __log2f(lsum)) * 0.69314718055994531f;
+  }
+}
+
 // F8 = 1: q and k arrive as FP8 E4M3 codes (one byte per element, d = 128: one
 // 128-byte swizzle row per token) and S = Q K^T runs as kind::f8f6f4 MMAs (K = 32
 // each); the host folds the two dequantisation scales into the softmax scale; P and V
@@ -300,6 +375,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   int head = blockIdx.y;
+  // key-range split (dense batches only): this CTA's share, = its rank in the cluster
+  const int n_split = p.kv_split > 1 ? p.kv_split : 1;
+  const int split = n_split > 1 ? static_cast<int>(blockIdx.x % n_split) : 0;
 
   // ---- work decode: which sequence, head and pair of query tiles
   int64_t seq_start, seq_len;
@@ -326,8 +404,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       rem -= np * p.H;
     }
   } else if (p.cu_seqlens == nullptr) {
-    const int seq = blockIdx.x / p.pairs_per_dense_seq;
-    pair = blockIdx.x - seq * p.pairs_per_dense_seq;
+    // head-major unit numbering: the (pairs, heads) grid's own block order
+    const int64_t per_head = static_cast<int64_t>(p.pairs_per_dense_seq) * p.n_seq;
+    const int64_t unit =
+        p.unit0 + (n_split > 1 ? static_cast<int64_t>(blockIdx.x / n_split)
+                               : static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x);
+    head = static_cast<int>(unit / per_head);
+    const int x = static_cast<int>(unit - static_cast<int64_t>(head) * per_head);
+    const int seq = x / p.pairs_per_dense_seq;
+    pair = x - seq * p.pairs_per_dense_seq;
     seq_len = p.dense_len;
     seq_start = static_cast<int64_t>(seq) * p.dense_len;
   } else {
@@ -350,6 +435,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int64_t q_row0 = static_cast<int64_t>(pair) * 2 * kTileM;  // within the sequence
   const int nk = static_cast<int>((seq_len + kTileN - 1) / kTileN);
   const int last_valid = static_cast<int>(seq_len - static_cast<int64_t>(nk - 1) * kTileN);
+  // key tiles [kb0, kb0 + nkl) of the nk (nk < 2^24, split < 8: int products); the
+  // loops below count j from 0 within them
+  const int kb0 = split * nk / n_split;
+  const int nkl = (split + 1) * nk / n_split - kb0;
+  // the last tile of the range is the sequence's ragged one
+  const bool ragged_last = kb0 + nkl == nk && last_valid < kTileN;
 
   Barriers* b = &bars;
   volatile int* abort = &s_abort;
@@ -406,7 +497,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float m = -INFINITY;  // running max of scale*log2(e)*score (lazily updated)
     uint64_t l2 = f2_pack(0.f, 0.f);  // running row sum, two partial sums
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
+    for (int j = 0; j < nkl; ++j) {
       // warp-uniform decision: tcgen05.ld/st below are warp-collective
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(bar_s, j & 1, abort, p.wait_limit_ns))) { ok = false; break; }
       ptx::tc_fence_after();
@@ -417,7 +508,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-      const bool ragged = j == nk - 1 && last_valid < kTileN;
+      const bool ragged = ragged_last && j == nkl - 1;
       if (ragged) {
 #pragma unroll
         for (int c = 0; c < 128; ++c)
@@ -510,8 +601,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float inv_l = p.o_scale / l;
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
                       ((seq_start + row_in_seq) * p.H + head) * static_cast<int64_t>(D) * 2;
+      if (n_split > 1) {
+        // a share of the keys: publish the unnormalised O row and (m, l) for the merge
+        const int g = qi * kTileM + r;
+        uint8_t* prow = smem + g * L::kPartStride;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(tO + c * 32, ov);
+          ptx::tmem_wait_ld();
+          uint4* dst = reinterpret_cast<uint4*>(prow + c * 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_uint4(ov[4 * e], ov[4 * e + 1], ov[4 * e + 2], ov[4 * e + 3]);
+        }
+        reinterpret_cast<float2*>(smem + L::kPartMl)[g] = make_float2(m, l);
+      }
+#pragma unroll 1
+      for (int c = 0; c < (n_split > 1 ? 0 : D / 32); ++c) {
         uint32_t ov[32];
         ptx::tmem_ld32(tO + c * 32, ov);
         ptx::tmem_wait_ld();
@@ -527,8 +634,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-      if (valid && p.lse != nullptr)
+      if (valid && n_split == 1 && p.lse != nullptr)
         p.lse[(seq_start + row_in_seq) * p.H + head] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+    if (n_split > 1) {
+      ptx::cluster_sync_all();  // every CTA of the cluster has published its partial rows
+      merge_split_rows<D>(smem, p, split, n_split, q_row0, seq_len, seq_start, head, tid);
+      ptx::cluster_sync_all();  // no CTA leaves while another may still read its memory
     }
   } else if (warp == kWarpTma || warp == kWarpTmaV) {
     // =========================================================== TMA producers
@@ -554,12 +666,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                x0 + blk * 64, static_cast<int>(seq_start + q_row0 + qi * kTileM),
                                q_full);
         }
-        for (int j = 0; j < nk; ++j) {
+        for (int j = 0; j < nkl; ++j) {
           const int st = j % stages;
           if (j >= stages &&
               !ptx::mbar_wait(ptx::smem_u32(&empty[st]), ((j / stages) - 1) & 1, abort, p.wait_limit_ns))
             break;
-          const int y = static_cast<int>(seq_start + static_cast<int64_t>(j) * kTileN);
+          const int y = static_cast<int>(seq_start + static_cast<int64_t>(kb0 + j) * kTileN);
           const uint32_t f = ptx::smem_u32(&full[st]);
           ptx::mbar_arrive_expect_tx(f, is_k ? kQKBytes : kVBytes);
           const int boxes = is_k ? kQKBoxes : kVBoxes;
@@ -659,10 +771,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (leader) ptx::umma_commit(ptx::smem_u32(&b->k_empty[0]));
         issued_any = true;
       }
-      for (int j = 0; ok && j < nk; ++j) {
+      for (int j = 0; ok && j < nkl; ++j) {
         const int vs = j % kVStages, vph = (j / kVStages) & 1;
         const int ks1 = (j + 1) % kKStages, kph1 = ((j + 1) / kKStages) & 1;
-        const bool more = j + 1 < nk;
+        const bool more = j + 1 < nkl;
         if (!(ok = wait(ptx::smem_u32(&b->v_full[vs]), vph))) break;
         if (!(ok = pv_tile(0, vs, j > 0, j))) break;
         if (more) {
@@ -713,11 +825,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         ptx::fence_proxy_async_smem();
         ptx::mbar_arrive(ptx::smem_u32(&b->q_ready));
-        for (int j = 0; j < nk; ++j) {
+        for (int j = 0; j < nkl; ++j) {
           const int st = j % kKStages, ph = (j / kKStages) & 1;
           if (!ptx::mbar_wait(ptx::smem_u32(&b->k_full[st]), ph, abort, p.wait_limit_ns)) break;
-          const int nv = (j == nk - 1) ? last_valid : kTileN;
-          rope_tile(smem + L::kK + st * L::kTile, static_cast<int64_t>(j) * kTileN, nv);
+          const int nv = (kb0 + j == nk - 1) ? last_valid : kTileN;
+          rope_tile(smem + L::kK + st * L::kTile, static_cast<int64_t>(kb0 + j) * kTileN, nv);
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(ptx::smem_u32(&b->k_ready[st]));
         }
@@ -725,6 +837,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   }
 
+  if (n_split > 1 && warp >= 8) {
+    // the two cluster barriers of the softmax warps' merge
+    ptx::cluster_sync_all();
+    ptx::cluster_sync_all();
+  }
   ptx::tc_fence_before();
   __syncthreads();
   if (tid == 0 && *abort) atomicOr(&g_device_error, kDevErrTimeout);

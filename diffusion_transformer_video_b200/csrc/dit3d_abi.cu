@@ -254,6 +254,64 @@ void set_seq_order(attn::Params* prm, const std::vector<int64_t>& lens, int64_t 
   prm->n_order = static_cast<int32_t>(order.size());
 }
 
+int dev_index() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev >= 0 && dev < 64 ? dev : 0;
+}
+int g_sm_count[64] = {};
+int g_last_attn_split = 0;  // key-range split of the last single-CTA attention launch
+
+// Key-range split of a dense attention launch's last partial wave. `units` = n_work * H
+// work units of one CTA each run in waves of one per SM; when the last wave holds
+// tail = units % SMs units, the SMs it leaves idle can share their work instead: every
+// tail unit becomes a cluster of S CTAs, each over nk / S of the key tiles, which merge
+// their partial results (attn_fwd_kernel, Params::kv_split). Returns the largest S in
+// [2, kMaxSplit] with tail * S CTAs within one wave, at least two key tiles per CTA, and
+// tail clusters of S resident at once (as the occupancy calculator reports for this
+// kernel, whose residency depends on D only); 1 (no split) when none qualifies.
+template <int D, typename Kernel>
+int attn_tail_split(Kernel kernel, uint32_t smem, const attn::Params& prm, int n_work, int32_t H) {
+  const int dev = dev_index();
+  if (g_sm_count[dev] == 0) {
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    g_sm_count[dev] = sms > 0 ? sms : 148;
+  }
+  const int64_t sms = g_sm_count[dev];
+  const int64_t units = static_cast<int64_t>(n_work) * H;
+  const int64_t tail = units % sms;
+  const int64_t nk = (prm.dense_len + attn::kTileN - 1) / attn::kTileN;
+  if (tail == 0) return 1;
+  // clusters of S resident at once, per S (0: not yet asked; -1: the query failed)
+  static int max_clusters[64][attn::kMaxSplit + 1] = {};
+  for (int S = attn::kMaxSplit; S >= 2; --S) {
+    if (tail * S > sms || 2 * S > nk) continue;
+    int& mc = max_clusters[dev][S];
+    if (mc == 0) {
+      cudaLaunchConfig_t cfg{};
+      cudaLaunchAttribute attr[1];
+      cfg.gridDim = dim3(static_cast<unsigned>(S));
+      cfg.blockDim = dim3(attn::kThreads);
+      cfg.dynamicSmemBytes = smem;
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();  // clear the query's error; the split is simply not used
+        n = -1;
+      }
+      mc = n;
+    }
+    if (mc > 0 && tail <= mc) return S;
+  }
+  return 1;
+}
+
 // F8: 0 all bf16; 1 E4M3 q and k; 2 E4M3 q, k and v (see attn_fwd_kernel)
 template <int D, int F8 = 0>
 int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32_t H,
@@ -275,9 +333,47 @@ int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32
       return DIT_ERR_LAUNCH;
     attr_set[dev] = true;
   }
-  // packed: 1-D grid over (sequence in prm.seq_order, head, pair); else (pairs, heads)
-  const dim3 grid = prm.n_order > 0 ? dim3(static_cast<unsigned>(n_work) * H) : dim3(n_work, H);
-  attn::attn_fwd_kernel<D, F8><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, prm);
+  attn::Params base = prm;
+  base.kv_split = 1;
+  base.unit0 = 0;
+  const int split = prm.cu_seqlens == nullptr && prm.n_order == 0
+                        ? attn_tail_split<D>(attn::attn_fwd_kernel<D, F8>, smem, prm, n_work, H)
+                        : 1;
+  g_last_attn_split = split;
+  if (split <= 1) {
+    // packed: 1-D grid over (sequence in prm.seq_order, head, pair); else (pairs, heads)
+    const dim3 grid = prm.n_order > 0 ? dim3(static_cast<unsigned>(n_work) * H) : dim3(n_work, H);
+    attn::attn_fwd_kernel<D, F8><<<grid, attn::kThreads, smem, stream>>>(tq, tk, tv, base);
+    return launch_status();
+  }
+  // dense batch whose last wave would run a few units on a mostly idle GPU: the whole
+  // waves as usual (1-D grid, head-major units), then the rest with each unit split
+  // over a cluster of `split` CTAs by key range
+  const int64_t units = static_cast<int64_t>(n_work) * H;
+  const int64_t tail = units % g_sm_count[dev_index()];
+  const int64_t full = units - tail;
+  if (full > 0) {
+    attn::attn_fwd_kernel<D, F8><<<static_cast<unsigned>(full), attn::kThreads, smem, stream>>>(
+        tq, tk, tv, base);
+    if (int s = launch_status()) return s;
+  }
+  attn::Params tp = base;
+  tp.kv_split = split;
+  tp.unit0 = static_cast<int32_t>(full);
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(tail * split));
+  cfg.blockDim = dim3(attn::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn::attn_fwd_kernel<D, F8>, tq, tk, tv, tp) != cudaSuccess)
+    return DIT_ERR_LAUNCH;
   return launch_status();
 }
 
@@ -915,6 +1011,8 @@ int dit_check_device(void* stream) {
 void dit_debug_force_timeout(int enable) { g_force_timeout = enable ? 1 : 0; }
 
 void dit_debug_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 2000000000ull; }
+
+int dit_debug_last_attn_split(void) { return g_last_attn_split; }
 
 int dit_set_attn_variant(int variant) {
   if (variant != 0 && variant != 1) return DIT_ERR_SHAPE;

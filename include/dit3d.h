@@ -194,6 +194,12 @@ int dit_rope3d_qk_e4m3(const void* q_in, const void* k_in, void* q8_out, void* k
  * are used as given. Rotating q and k first with dit_rope3d_qk and passing NULL
  * gives the same bits and is faster on long sequences (in-kernel, every K tile is
  * rotated again for each pair of query tiles); the in-kernel form needs no scratch.
+ * Dense batches (cu_seqlens NULL) whose last wave of work units (a pair of 128-row
+ * query tiles of one sequence and head, one CTA per SM) would leave most SMs idle run
+ * that wave split by key range: each of those units is a cluster of 2-8 CTAs that
+ * each take a share of the key tiles and merge their partial results through
+ * distributed shared memory (no scratch memory). Such units differ from the unsplit
+ * form only in rounding (the same online-softmax rescaling, applied across shares).
  *   q, k, v, o : [rows, H, d] bf16, o must not overlap q, k or v
  *   lse        : NULL or [rows, H] fp32, natural-log sum of exp(scale * scores)
  *   softmax_scale <= 0 selects 1/sqrt(d).
@@ -326,6 +332,13 @@ void dit_debug_force_timeout(int enable);
  * dit_check_device() returns as DIT_ERR_TIMEOUT. The CTA-pair kernels keep 2 s. A plain
  * process-wide setting, not synchronised. */
 void dit_debug_wait_limit_ns(uint64_t ns);
+
+/* Test hook: the number of CTAs each work unit of the last single-CTA attention launch
+ * (dit_attn_fwd, dit_attn_fwd_noalloc, dit_attn_fwd_qk8, dit_attn_fwd_fp8 with
+ * variant 0) was split over by key range: 1 for no split, 2-8 when a dense batch's last
+ * partial wave ran as clusters that merge their partial results (see dit_attn_fwd), 0
+ * before any launch. Not synchronised between threads. */
+int dit_debug_last_attn_split(void);
 
 #ifdef __cplusplus
 }

@@ -84,6 +84,18 @@ def test_guards_survive_every_kernel():
     dit3d.dit_check_device()
     checks += [("quantize", _intact(cb, codes.numel())), ("fp8 attention", _intact(fb, fo.numel()))]
 
+    # dense rows whose units run split by key range (clusters merging partial results)
+    rs = 1100                                     # a last query-tile pair with one empty tile
+    qs, ks, vs = bf(rs, H, d), bf(rs, H, d), bf(rs, H, d)
+    sb, so = _guarded((rs, H, d), torch.bfloat16)
+    slb, sl = _guarded((rs, H), torch.float32)
+    assert L.dit_attn_fwd(ctypes.c_void_p(qs.data_ptr()), ctypes.c_void_p(ks.data_ptr()),
+                          ctypes.c_void_p(vs.data_ptr()), ctypes.c_void_p(so.data_ptr()),
+                          ctypes.c_void_p(sl.data_ptr()), rs, H, d, 1, None, None, 0.0, None, st) == 0
+    dit3d.dit_check_device()
+    assert L.dit_debug_last_attn_split() >= 2
+    checks += [("split attention", _intact(sb, so.numel())), ("split lse", _intact(slb, sl.numel()))]
+
     bad = [name for name, ok in checks if not ok]
     assert not bad, f"guard regions overwritten by: {bad}"
 
