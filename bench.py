@@ -599,7 +599,6 @@ def main():
                              "bytes_equal_two_pass": bool(torch.equal(q8f, q8) and torch.equal(k8f, k8)),
                              "kernel": "dit_rope3d_qk_e4m3 (RoPE and E4M3 in one pass)"},
                "in_step": False, "note": "E4M3 q, k (scale 1/64), bf16 P and V"}
-        del q8f, k8f
         # all of q, k, v (and P) in E4M3
         v8 = dit3d.dit_quantize_e4m3(dev["v"], 64.0)
         for _ in range(2):
@@ -618,7 +617,43 @@ def main():
         fp8["all_fp8"] = {"ms": t_f8, "TFLOP/s": w.attn_flops() / (t_f8 * 1e-3) / 1e12,
                           "max_abs_vs_bf16_attention": float((o8.float() - o.float()).abs().max()),
                           "note": "E4M3 q, k, v and P"}
-        del q8, k8, v8, o8
+
+        # the block's step with E4M3 attention operands, timed on its own: modulate ->
+        # RoPE with E4M3 output -> attention (E4M3 Q K^T; or all E4M3, v quantised in the
+        # step) -> gated residual
+        prm0 = run.params[0]
+        x_out = torch.empty_like(dev["x"])
+
+        def fp8_step(all8):
+            dit3d.dit_adaln_modulate(dev["x"], prm0["gamma"], prm0["beta"], rpg, out=u)
+            dit3d.dit_rope3d_qk_e4m3(dev["q"], dev["k"], run.desc, 64.0, 64.0, n_seq=w.n_seq,
+                                     cu_seqlens=cu, q8_out=q8f, k8_out=k8f)
+            if all8:
+                dit3d.dit_quantize_e4m3(dev["v"], 64.0, out=v8)
+                dit3d.dit_attn_fwd_fp8(q8f, k8f, v8, 1 / 64, 1 / 64, 1 / 64, n_seq=w.n_seq,
+                                       cu_seqlens=cu, out=o8)
+            else:
+                dit3d.dit_attn_fwd_qk8(q8f, k8f, dev["v"], 1 / 64, 1 / 64, n_seq=w.n_seq,
+                                       cu_seqlens=cu, out=o8)
+            dit3d.dit_gated_residual(dev["x"], o8.view(rows, D), prm0["alpha"], rpg, out=x_out)
+
+        for all8, key in ((False, "step_qk8"), (True, "step_all_fp8")):
+            for _ in range(3):
+                fp8_step(all8)
+            ev6 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(max(K, 3))]
+            for a, b in ev6:
+                a.record(stream)
+                fp8_step(all8)
+                b.record(stream)
+            torch.cuda.synchronize()
+            dit3d.dit_check_device()
+            t_s = statistics.mean(a.elapsed_time(b) for a, b in ev6)
+            fp8[key] = {"ms": t_s, "TFLOP/s": w.attn_flops() / (t_s * 1e-3) / 1e12,
+                        "calls": "dit_adaln_modulate, dit_rope3d_qk_e4m3, "
+                                 + ("dit_quantize_e4m3 (v), dit_attn_fwd_fp8" if all8
+                                    else "dit_attn_fwd_qk8") + ", dit_gated_residual"}
+        del q8, k8, v8, o8, q8f, k8f, x_out
 
     # the block's linear layers (projections with the fused adaLN-Zero gate, MLP up with
     # GELU), timed on their own: not part of the step; cuBLAS on the same shapes for context

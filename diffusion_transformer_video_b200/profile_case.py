@@ -27,6 +27,7 @@ def main():
     ap.add_argument("--d-model", type=int, default=0, help="activation width (modulate, residual, euler)")
     ap.add_argument("--heads", type=int, default=0)
     ap.add_argument("--head-dim", type=int, default=128)
+    ap.add_argument("--n-seq", type=int, default=1, help="attention: equal dense sequences")
     ap.add_argument("--rows-per-group", type=int, default=0, help="default: every row one group")
     ap.add_argument("--grid", type=int, nargs=2, default=(30, 52), help="patch grid (RoPE)")
     ap.add_argument("--bands", type=int, nargs=3, default=(44, 42, 42))
@@ -64,7 +65,9 @@ def main():
             o = torch.empty_like(q)
             # attn_rope: q and k rotated inside the attention kernel (fused 3D-RoPE)
             rope = desc if a.kernel == "attn_rope" else None
-            call = lambda: dit3d.dit_attn_fwd(q, k, v, out=o, rope=rope)
+            if rows % a.n_seq:
+                raise SystemExit(f"rows must split into {a.n_seq} equal sequences")
+            call = lambda: dit3d.dit_attn_fwd(q, k, v, n_seq=a.n_seq, out=o, rope=rope)
     else:
         K, N = D, a.n_out or 3 * D
         x, w = bf(rows, K), bf(N, K, std=K ** -0.5)
