@@ -39,12 +39,13 @@ sys.path.insert(0, ROOT)
 METRIC = "3D-RoPE attention TFLOP/s & % BF16 peak; adaLN GB/s & % HBM peak (1xB200)"
 UNIT = "TFLOP/s"
 # DRAM bytes per head of one attention launch at the 480P geometry, from an ncu capture
-# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum = 406.48 + 117.93 MB, over
-# 16; with in-kernel RoPE 407.39 + 119.45 MB), keyed by RoPE mode ("prepass" and "none"
-# run the same kernel, without in-kernel RoPE). Heads are independent, so a launch's
-# traffic is this times its head count. Other workloads report null.
-ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 524.411392e6 / 16, "none": 524.411392e6 / 16,
-                                 "fused": 526.841856e6 / 16}
+# with 16 heads (dram__bytes_read.sum + dram__bytes_write.sum = 410.445 + 118.815 MB, over
+# 16), keyed by RoPE mode ("prepass" and "none" run the same kernel, without in-kernel
+# RoPE; the in-kernel RoPE mode has no capture of the current kernel: null). Heads are
+# independent, so a launch's traffic is this times its head count. Other workloads
+# report null.
+ATTN_DRAM_BYTES_PER_HEAD_480P = {"prepass": 529.260544e6 / 16, "none": 529.260544e6 / 16,
+                                 "fused": None}
 
 
 def _peaks():
