@@ -262,14 +262,30 @@ int dev_index() {
 int g_sm_count[64] = {};
 int g_last_attn_split = 0;  // key-range split of the last single-CTA attention launch
 
-// Key-range split of a dense attention launch's last partial wave. `units` = n_work * H
-// work units of one CTA each run in waves of one per SM; when the last wave holds
-// tail = units % SMs units, the SMs it leaves idle can share their work instead: every
+// Key-range split of a dense attention launch's last partial wave. `units` work units
+// of one CTA each run in waves of one per SM; when the last wave holds
+// tail = units % sms units, the SMs it leaves idle can share their work instead: every
 // tail unit becomes a cluster of S CTAs, each over nk / S of the key tiles, which merge
 // their partial results (attn_fwd_kernel, Params::kv_split). Returns the largest S in
 // [2, kMaxSplit] with tail * S CTAs within one wave, at least two key tiles per CTA, and
-// tail clusters of S resident at once (as the occupancy calculator reports for this
-// kernel, whose residency depends on D only); 1 (no split) when none qualifies.
+// tail clusters of S resident at once (resident(S): the occupancy calculator's count,
+// asked only for the S values that pass the first two tests); 1 (no split) when none
+// qualifies.
+template <typename Resident>
+int tail_split_choice(int64_t units, int64_t sms, int64_t nk, Resident resident) {
+  if (sms <= 0 || units <= 0) return 1;
+  const int64_t tail = units % sms;
+  if (tail == 0) return 1;
+  for (int S = attn::kMaxSplit; S >= 2; --S) {
+    if (tail * S > sms || 2 * S > nk) continue;
+    const int mc = resident(S);
+    if (mc > 0 && tail <= mc) return S;
+  }
+  return 1;
+}
+
+// tail_split_choice for a launch of this kernel (whose residency depends on D only) on
+// the current device.
 template <int D, typename Kernel>
 int attn_tail_split(Kernel kernel, uint32_t smem, const attn::Params& prm, int n_work, int32_t H) {
   const int dev = dev_index();
@@ -278,15 +294,11 @@ int attn_tail_split(Kernel kernel, uint32_t smem, const attn::Params& prm, int n
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     g_sm_count[dev] = sms > 0 ? sms : 148;
   }
-  const int64_t sms = g_sm_count[dev];
   const int64_t units = static_cast<int64_t>(n_work) * H;
-  const int64_t tail = units % sms;
   const int64_t nk = (prm.dense_len + attn::kTileN - 1) / attn::kTileN;
-  if (tail == 0) return 1;
   // clusters of S resident at once, per S (0: not yet asked; -1: the query failed)
   static int max_clusters[64][attn::kMaxSplit + 1] = {};
-  for (int S = attn::kMaxSplit; S >= 2; --S) {
-    if (tail * S > sms || 2 * S > nk) continue;
+  return tail_split_choice(units, g_sm_count[dev], nk, [&](int S) {
     int& mc = max_clusters[dev][S];
     if (mc == 0) {
       cudaLaunchConfig_t cfg{};
@@ -307,9 +319,8 @@ int attn_tail_split(Kernel kernel, uint32_t smem, const attn::Params& prm, int n
       }
       mc = n;
     }
-    if (mc > 0 && tail <= mc) return S;
-  }
-  return 1;
+    return mc;
+  });
 }
 
 // F8: 0 all bf16; 1 E4M3 q and k; 2 E4M3 q, k and v (see attn_fwd_kernel)
@@ -1013,6 +1024,13 @@ void dit_debug_force_timeout(int enable) { g_force_timeout = enable ? 1 : 0; }
 void dit_debug_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns ? ns : 2000000000ull; }
 
 int dit_debug_last_attn_split(void) { return g_last_attn_split; }
+
+int dit_debug_tail_split(int64_t units, int64_t sms, int64_t nk, const int32_t* resident,
+                         int32_t* split) {
+  if (resident == nullptr || split == nullptr) return DIT_ERR_NULL;
+  *split = tail_split_choice(units, sms, nk, [&](int S) { return static_cast<int>(resident[S]); });
+  return DIT_OK;
+}
 
 int dit_set_attn_variant(int variant) {
   if (variant != 0 && variant != 1) return DIT_ERR_SHAPE;

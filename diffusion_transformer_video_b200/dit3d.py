@@ -28,7 +28,7 @@ EXPORTS = ("dit_adaln_modulate", "dit_gated_residual", "dit_flow_euler_step", "d
            "dit_attn_fwd_noalloc", "dit_check_device", "dit_status_string", "dit_shutdown",
            "dit_set_attn_variant", "dit_debug_force_timeout",
            "dit_debug_wait_limit_ns", "dit_wait_device", "dit_debug_poll_fake", "dit_debug_exp2_fma",
-           "dit_debug_last_attn_split")
+           "dit_debug_last_attn_split", "dit_debug_tail_split")
 
 
 class DitError(RuntimeError):
@@ -96,6 +96,7 @@ def lib():
         L.dit_debug_poll_fake.restype = ctypes.c_int
         L.dit_debug_exp2_fma.argtypes = [P, P, i64, P]
         L.dit_debug_last_attn_split.argtypes = []
+        L.dit_debug_tail_split.argtypes = [i64, i64, i64, P, P]
         L.dit_debug_exp2_fma.restype = ctypes.c_int
         for name in ("dit_adaln_modulate", "dit_gated_residual", "dit_rope3d_qk", "dit_attn_fwd",
                      "dit_check_device"):

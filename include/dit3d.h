@@ -340,6 +340,15 @@ void dit_debug_wait_limit_ns(uint64_t ns);
  * before any launch. Not synchronised between threads. */
 int dit_debug_last_attn_split(void);
 
+/* Test hook of the split rule above, on the host with made-up figures (needs no GPU):
+ * writes to *split the split S (1 = none) for `units` work units, `sms` SMs and `nk` key
+ * tiles per unit, where resident[S] (S = 0..8) stands for the number of clusters of S
+ * CTAs that fit at once: the largest S in 2..8 with (units % sms) * S <= sms,
+ * 2 * S <= nk and resident[S] >= units % sms; 1 when units % sms == 0 or none
+ * qualifies. Errors: DIT_ERR_NULL for a NULL `resident` or `split`. */
+int dit_debug_tail_split(int64_t units, int64_t sms, int64_t nk, const int32_t* resident,
+                         int32_t* split);
+
 #ifdef __cplusplus
 }
 #endif

@@ -95,6 +95,29 @@ def test_validation_before_any_device_work(L):
     assert e4(FAKE, k_in, apart, None) == 1
 
 
+def test_tail_split_rule(L):
+    # the split of a dense attention launch's last partial wave, on made-up residency
+    def split(units, sms, nk, resident):
+        arr = (ctypes.c_int32 * 9)(*resident)
+        out = ctypes.c_int32(-7)
+        assert L.dit_debug_tail_split(units, sms, nk, arr, ctypes.byref(out)) == 0
+        return out.value
+    fits = [0, 0, 74, 49, 37, 29, 24, 21, 18]          # every size fits its tail
+    # image: 768 units on 148 SMs -> 28 left: 5 x 28 = 140 CTAs, or 4 when 5 does not fit
+    assert split(768, 148, 32, fits) == 5
+    assert split(768, 148, 32, [0, 0, 74, 49, 37, 24, 24, 21, 18]) == 4
+    assert split(5120, 148, 256, fits) == 1               # 480P: 88 left, 2 x 88 > 148
+    assert split(8560, 148, 214, fits) == 1               # 720P: 124 left
+    assert split(740, 148, 32, fits) == 1                 # whole waves only
+    assert split(16, 148, 32, [0, 0, 74, 49, 37, 29, 24, 21, 18]) == 8   # one small wave
+    assert split(16, 148, 6, fits) == 3                   # two key tiles per share at least
+    assert split(16, 148, 3, fits) == 1                   # too few key tiles to share
+    assert split(24, 148, 8, fits) == 4                   # 6 fits the wave, not 8 key tiles
+    assert split(28, 148, 32, [0, 0, -1, -1, -1, -1, -1, -1, -1]) == 1   # residency unknown
+    out = ctypes.c_int32(0)
+    assert L.dit_debug_tail_split(768, 148, 32, None, ctypes.byref(out)) == 1   # DIT_ERR_NULL
+
+
 @pytest.mark.skipif(os.environ.get("CUDA_VISIBLE_DEVICES", None) is None and
                     not os.path.exists("/dev/nvidia0") is False, reason="GPU present")
 def test_valid_call_without_gpu_reports_device_error(L):
