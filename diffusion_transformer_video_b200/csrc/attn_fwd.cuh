@@ -88,6 +88,10 @@ struct Params {
   // results through distributed shared memory (the launch's last partial wave)
   int32_t kv_split;
   int32_t unit0;
+  // programmatic dependent launch of the split wave: 1 = let the next launch (the split
+  // units) start as this grid's CTAs are all resident; 2 = wait, before exiting, for the
+  // launch this one overlaps, so that later work on the stream still follows both
+  int32_t pdl;
 };
 constexpr int kMaxOrder = 64;
 constexpr int kMaxSplit = 8;  // portable cluster size
@@ -375,6 +379,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   int head = blockIdx.y;
+  if (p.pdl & 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // key-range split (dense batches only): this CTA's share, = its rank in the cluster
   const int n_split = p.kv_split > 1 ? p.kv_split : 1;
   const int split = n_split > 1 ? static_cast<int>(blockIdx.x % n_split) : 0;
@@ -849,6 +854,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
+  if ((p.pdl & 2) && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace attn

@@ -347,6 +347,7 @@ int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32
   attn::Params base = prm;
   base.kv_split = 1;
   base.unit0 = 0;
+  base.pdl = 0;
   const int split = prm.cu_seqlens == nullptr && prm.n_order == 0
                         ? attn_tail_split<D>(attn::attn_fwd_kernel<D, F8>, smem, prm, n_work, H)
                         : 1;
@@ -364,15 +365,19 @@ int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32
   const int64_t tail = units % g_sm_count[dev_index()];
   const int64_t full = units - tail;
   if (full > 0) {
+    // the split units may start on SMs as the whole waves drain (they read only q, k, v)
+    attn::Params mp = base;
+    mp.pdl = 1;
     attn::attn_fwd_kernel<D, F8><<<static_cast<unsigned>(full), attn::kThreads, smem, stream>>>(
-        tq, tk, tv, base);
+        tq, tk, tv, mp);
     if (int s = launch_status()) return s;
   }
   attn::Params tp = base;
   tp.kv_split = split;
   tp.unit0 = static_cast<int32_t>(full);
+  tp.pdl = full > 0 ? 2 : 0;
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(static_cast<unsigned>(tail * split));
   cfg.blockDim = dim3(attn::kThreads);
   cfg.dynamicSmemBytes = smem;
@@ -381,8 +386,12 @@ int launch_attn(const void* q, const void* k, const void* v, int64_t rows, int32
   attr[0].val.clusterDim.x = static_cast<unsigned>(split);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // overlap only the launch just made above: with no whole waves before it, the split
+  // launch follows the stream's previous work in the usual order
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = full > 0 ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, attn::attn_fwd_kernel<D, F8>, tq, tk, tv, tp) != cudaSuccess)
     return DIT_ERR_LAUNCH;
   return launch_status();
