@@ -29,7 +29,10 @@
  *    cos/sin tables (angles in fp64, stored fp32, written by a kernel) are cached in
  *    device memory per (device, descriptor, extent) on first use and freed by
  *    dit_shutdown(). The first call for a given RoPE descriptor allocates and waits for
- *    its table: make it outside CUDA-graph capture.
+ *    its table: make it outside CUDA-graph capture. Likewise the first attention call
+ *    on a device whose dense batch gets its last wave split (see dit_attn_fwd) asks
+ *    the occupancy calculator how many clusters fit, once per cluster size; make a
+ *    call of the same shape before capturing one.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls only enqueue
  *    work: they return before the GPU has run it. Validation reads host data only.
  *  - Return value: DIT_OK or a dit_status code; nothing is printed, thrown or
