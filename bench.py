@@ -151,10 +151,37 @@ def cpu_oracle_attention(w, qkv64, n_rows: int, seed: int = 0):
     cpu_oracle_attention.last = (rows, ref_o)  # kept for the parity figures of the GPU arm
     seq_of = np.searchsorted(cu, rows, side="right") - 1
     flops = float(sum(4.0 * (cu[s + 1] - cu[s]) * w.head_dim * w.heads for s in seq_of))
-    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    threads = oracle.threads()
     sample = (f"{n_rows} query rows x {w.heads} heads of {w.name}, all keys of their sequence; "
               f"the oracle's 3D-RoPE of the full q and k is inside the timed call (fp64, OpenMP)")
     return flops / dt / 1e12, dt, sample, threads
+
+
+def cpu_oracle_attention_one_thread(w, qkv64, n_rows: int, seed: int = 0):
+    """The oracle's attention on one host thread, over operands it rotated beforehand
+    on all threads (its fp64 3D-RoPE of the whole q and k would dominate a one-thread
+    sample): TFLOP/s, seconds and the sample, for `n_rows` sampled query rows."""
+    import oracle
+    rng = np.random.default_rng([seed, 78])
+    rows = np.sort(rng.choice(w.rows, size=n_rows, replace=False)).astype(np.int64)
+    cu = w.cu_seqlens
+    q, k, v = qkv64
+    r = w.rope_desc()
+    qr = oracle.rope3d(q, cu, r["grid_h"], r["grid_w"], r["bands"], r["base"], r["offsets"])
+    kr = oracle.rope3d(k, cu, r["grid_h"], r["grid_w"], r["bands"], r["base"], r["offsets"])
+    before = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.attn_fwd(qr, kr, v, cu, qrows=rows)
+        dt = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(before)
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+    flops = float(sum(4.0 * (cu[s + 1] - cu[s]) * w.head_dim * w.heads for s in seq_of))
+    sample = (f"{n_rows} query rows x {w.heads} heads of {w.name}, all keys of their sequence, "
+              f"q and k rotated before the timed call (fp64, 1 thread)")
+    return flops / dt / 1e12, dt, sample
 
 
 L2_BYTES = 126e6                    # B200 L2
@@ -804,9 +831,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tf, dt, sample, threads = cpu_oracle_attention(w, widen_qkv(inp), args.cpu_rows, args.seed)
+        qkv64 = widen_qkv(inp)
+        tf, dt, sample, threads = cpu_oracle_attention(w, qkv64, args.cpu_rows, args.seed)
         cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
                "seconds": dt}
+        tf1, dt1, sample1 = cpu_oracle_attention_one_thread(w, qkv64, max(4, args.cpu_rows // 8),
+                                                            args.seed)
+        del qkv64
+        cpu["one_thread"] = {"value": tf1, "unit": UNIT, "cores": 1, "seconds": dt1,
+                             "sample": sample1}
         # the step's attention output on the same sampled rows, against the oracle
         run.step(i=0)
         s_rows, ref_o = cpu_oracle_attention.last

@@ -64,12 +64,26 @@ def _load():
         lib.oracle_rope3d.argtypes = [P, P, i64, i32, i32, P, i32, i32, i32, i32, i32, i32, f64,
                                       i32, i32, i32]
         lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, i64, i32, i32, P, i32, f64, P, i64]
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = ctypes.c_int
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = None
         for f in (lib.oracle_adaln_modulate, lib.oracle_gated_residual, lib.oracle_rope3d,
                   lib.oracle_attn_fwd, lib.oracle_flow_euler_step, lib.oracle_linear,
                   lib.oracle_quantize_e4m3, lib.oracle_round_bf16):
             f.restype = None
         _lib = lib
     return _lib
+
+
+def threads() -> int:
+    """Threads the oracle's OpenMP loops run on."""
+    return int(_load().oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """Run the oracle's OpenMP loops on n threads from now on."""
+    _load().oracle_set_threads(int(n))
 
 
 def _f64(a) -> np.ndarray:

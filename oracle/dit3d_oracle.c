@@ -26,6 +26,28 @@
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* The number of threads the OpenMP loops below run on (1 without OpenMP), and a way
+ * to set it, so that a timing of the oracle can state the host cores it used. No
+ * arithmetic of the method. */
+int oracle_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
 
 /* Token j of a sequence laid out row-major over the patch grid (t slowest, w
  * fastest): recover its (t, h, w) patch coordinates. Reading: the pages give
