@@ -39,6 +39,12 @@
 // which keeps every exponent <= 8 and skips most O rescales.
 // Every mbarrier wait is bounded; on expiry the CTA sets an error bit, drains its
 // in-flight copies and MMAs, frees its tensor memory and exits.
+// Key-range split (Params::kv_split > 1, the last partial wave of a dense batch): the
+// CTAs of a cluster share one unit's key tiles; each leaves its unnormalised O rows and
+// (m, l) in its own shared memory, and after a cluster barrier merges a share of the
+// unit's rows from every CTA's (merge_split_rows); a second barrier keeps each CTA's
+// memory alive until its peers have read it. Every path, bounded-wait expiry included,
+// reaches both barriers.
 #pragma once
 #include <type_traits>
 #include "common.cuh"
