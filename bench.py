@@ -157,6 +157,31 @@ def cpu_oracle_attention(w, qkv64, n_rows: int, seed: int = 0):
     return flops / dt / 1e12, dt, sample, threads
 
 
+def cpu_oracle_memory_steps(w, x_bits, seed: int = 0, n_rows: int = 4096):
+    """The oracle's adaLN modulation and gated residual on the first `n_rows` rows of
+    x (one parameter group; the residual's branch input y is the next `n_rows` rows of
+    x), on all its threads. Rates are in the bf16 algorithmic bytes of the GPU kernels
+    (4 and 6 bytes per element), so that they compare with the GPU figures."""
+    import oracle
+    from diffusion_transformer_video_b200 import workloads as wl
+    n = min(n_rows, w.rows // 2)
+    D = w.d_model
+    x = wl.bf16_bits_to_f64(x_bits[:n])
+    y = wl.bf16_bits_to_f64(x_bits[n:2 * n])
+    prm = wl.make_inputs(w, seed, which=("gamma", "beta", "alpha"))
+    g, b, a = (wl.bf16_bits_to_f64(prm[k][:1]) for k in ("gamma", "beta", "alpha"))
+    out = {}
+    for name, call, per_elem in (("adaln_modulate", lambda: oracle.adaln_modulate(x, g, b, n), 4),
+                                 ("gated_residual", lambda: oracle.gated_residual(x, y, a, n), 6)):
+        t0 = time.perf_counter()
+        call()
+        dt = time.perf_counter() - t0
+        out[name] = {"GB/s": per_elem * n * D / dt / 1e9, "seconds": dt, "rows": n}
+    out["sample"] = (f"the first {n} rows x {D} of {w.name}'s x (the residual's y: the next "
+                     f"{n}), one parameter group, fp64, {oracle.threads()} threads")
+    return out
+
+
 def cpu_oracle_attention_one_thread(w, qkv64, n_rows: int, seed: int = 0):
     """The oracle's attention on one host thread, over operands it rotated beforehand
     on all threads (its fp64 3D-RoPE of the whole q and k would dominate a one-thread
@@ -840,6 +865,7 @@ def main():
         del qkv64
         cpu["one_thread"] = {"value": tf1, "unit": UNIT, "cores": 1, "seconds": dt1,
                              "sample": sample1}
+        cpu["memory_steps"] = cpu_oracle_memory_steps(w, inp["x"], args.seed)
         # the step's attention output on the same sampled rows, against the oracle
         run.step(i=0)
         s_rows, ref_o = cpu_oracle_attention.last

@@ -60,3 +60,12 @@ def test_clock_summary_reports_reasons_power_and_the_active_mask(tmp_path):
     assert s["sm_mhz"] == 1605 and s["sm_max_mhz"] == 1965
     assert s["reasons"] == ["sw_power_cap"] and s["active_mask"] == "0x4"
     assert s["power_w"] == 996.0 and s["samples"] == 4
+
+
+def test_oracle_memory_steps_baseline_on_the_tiny_workload():
+    w = wl.get_workload("tiny")
+    x = wl.make_inputs(w, seed=0, which=("x",))["x"]
+    r = bench.cpu_oracle_memory_steps(w, x, 0)
+    for name in ("adaln_modulate", "gated_residual"):
+        assert r[name]["GB/s"] > 0 and r[name]["rows"] == w.rows // 2
+    assert "threads" in r["sample"]
