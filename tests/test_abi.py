@@ -144,3 +144,16 @@ def test_watchdog_poll_loop_with_a_fake_query(L):
     assert L.dit_debug_poll_fake(0, 0, 0, None) == 0        # done at the first poll
     assert L.dit_debug_poll_fake(5, 0, 0, None) == 7        # no time allowed
     assert L.dit_wait_device(None, -1) == 2                 # rejected before any CUDA call
+
+
+def test_every_declaration_has_its_own_doc_comment():
+    # each function the header declares is directly preceded by its own /* ... */ block
+    lines = open(os.path.join(ROOT, "include", "dit3d.h")).read().splitlines()
+    for i, line in enumerate(lines):
+        m = re.match(r"^(?:int|void|const char\*)\s+(dit_[a-z0-9_]+)\(", line)
+        if not m:
+            continue
+        j = i - 1
+        while j >= 0 and lines[j].strip() == "":
+            j -= 1
+        assert lines[j].rstrip().endswith("*/"), f"{m.group(1)} has no doc comment right above it"
